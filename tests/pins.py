@@ -1,0 +1,396 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each pin is a plain function that raises AssertionError on a mismatch.  The
+pins use hand-worked fixtures (tests/golden), closed forms, invariants,
+brute force by set enumeration, and library routines (torch fp64 softmax /
+scaled_dot_product_attention) for the special cases that reduce to them.
+test_oracle_pins.py runs them on the oracle; test_oracle_mutants.py runs them
+on builds of the oracle with planted mistakes and expects each to be caught.
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+from trainable_block_sparse_mean_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line.split()
+
+
+def _bf16(x) -> np.ndarray:
+    return synth.bf16_bits(np.asarray(x, np.float32))
+
+
+def _f64(b) -> np.ndarray:
+    return synth.bf16_to_f32(b).astype(np.float64)
+
+
+def _shape(**kw) -> synth.Shape:
+    return synth.Shape(**kw)
+
+
+# --------------------------------------------------------------------------
+# stage 1: mean pooling of K
+# --------------------------------------------------------------------------
+
+def pin_compress_hand():
+    sh = _shape(n=64, h_q=1, h_kv=1, d=2)
+    p = oracle.params(sh)
+    t = np.arange(64, dtype=np.float32)
+    k = _bf16(np.stack([t, -t / 2], axis=1)[:, None, :])
+    kc1 = _f64(oracle.compress_k(p, k))
+    assert kc1.shape == (3, 1, 2), kc1.shape
+    for j, c, val in _lines("compress_hand.txt"):
+        assert kc1[int(j), 0, int(c)] == float(val), (j, c, kc1[int(j), 0, int(c)], val)
+
+
+def pin_compress_ties():
+    sh = _shape(n=32, h_q=1, h_kv=1, d=1)
+    p = oracle.params(sh)
+    for odd, exact, want in _lines("compress_ties.txt"):
+        col = np.ones(32, np.float32)
+        col[7] = float(odd)
+        k = _bf16(col[:, None, None])
+        got = _f64(oracle.compress_k(p, k))[0, 0, 0]
+        assert float(Fraction(float(odd)) + 31) / 32 == float(exact)
+        assert got == float(want), (odd, got, want)
+
+
+def pin_compress_constant_and_ramp():
+    sh = _shape(n=200, h_q=2, h_kv=2, d=4)
+    p = oracle.params(sh)
+    c = np.array([0.375, -2.5, 7.0, 1e-3], np.float32)
+    k = np.zeros((200, 2, 4), np.float32)
+    k[:, 0, :] = c
+    k[:, 1, :] = (np.arange(200, dtype=np.float32) * 0.25)[:, None]
+    kb = _bf16(k)
+    kc1 = _f64(oracle.compress_k(p, kb))
+    nc = (200 - 32) // 16 + 1
+    assert kc1.shape[0] == nc
+    cb = _f64(_bf16(c))
+    for j in range(nc):
+        assert np.array_equal(kc1[j, 0], cb), (j, kc1[j, 0])
+        # ramp 0.25*t over tokens 16j..16j+31 -> 0.25*(16j + 15.5), exact in bf16 here
+        mid = 0.25 * (16 * j + 15.5)
+        assert np.all(kc1[j, 1] == _f64(_bf16(np.float32(mid)))), (j, kc1[j, 1], mid)
+
+
+def _rne_bf16_fraction(x: Fraction) -> float:
+    """Nearest bf16 value to the exact rational x, ties to even (brute force)."""
+    if x == 0:
+        return 0.0
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = 0
+    while a >= 2:
+        a /= 2
+        e += 1
+    while a < 1:
+        a *= 2
+        e -= 1
+    q = max(e - 7, -133)
+    scaled = abs(x) / Fraction(2) ** q
+    lo = scaled.numerator // scaled.denominator
+    rem = scaled - lo
+    r = lo + 1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1) else lo
+    return sign * float(Fraction(r) * Fraction(2) ** q)
+
+
+def pin_compress_bruteforce():
+    sh = _shape(n=96, h_q=2, h_kv=2, d=8)
+    p = oracle.params(sh)
+    rng = np.random.default_rng(11)
+    k = _bf16(rng.standard_normal((96, 2, 8)).astype(np.float32) * 3)
+    kv = _f64(k)
+    kc1 = _f64(oracle.compress_k(p, k))
+    nc = (96 - 32) // 16 + 1
+    assert kc1.shape == (nc, 2, 8)
+    for j in range(nc):
+        for g in range(2):
+            for c in range(8):
+                s = sum(Fraction(float(kv[t, g, c])) for t in range(16 * j, 16 * j + 32))
+                want = _rne_bf16_fraction(s / 32)
+                assert kc1[j, g, c] == want, (j, g, c, kc1[j, g, c], want)
+
+
+def pin_visibility():
+    p = oracle.params(_shape())
+    for n in range(0, 140):
+        want = sum(1 for j in range(n) if 16 * j + 32 <= n)
+        assert oracle.num_kernels(p, n) == want, (n,)
+    for i in range(0, 200):
+        # kernel j covers tokens 16j..16j+31; visible to query i if all <= i
+        want = sum(1 for j in range(i + 1) if set(range(16 * j, 16 * j + 32)) <= set(range(i + 1)))
+        assert oracle.visible_kernels(p, i) == want, (i,)
+
+
+# --------------------------------------------------------------------------
+# stage 2: S^C1 softmax and the group sum S^shared
+# --------------------------------------------------------------------------
+
+def _small_problem(n=300, h_q=4, h_kv=2, d=16, seed=5, **kw):
+    sh = _shape(n=n, h_q=h_q, h_kv=h_kv, d=d, **kw)
+    data = synth.make_prefill(sh, seed=seed)
+    return sh, data
+
+
+def pin_scores_sum_to_G():
+    sh, data = _small_problem()
+    p = oracle.params(sh)
+    kc1 = oracle.compress_k(p, data["k"])
+    for i in (31, 47, 120, 299):
+        for g in range(sh.h_kv):
+            s, _ = oracle.shared_scores_row(p, data["q"], kc1, i, g)
+            assert abs(s.sum() - sh.G) < 1e-12, (i, g, s.sum())
+            assert np.all(s > 0)
+
+
+def pin_scores_uniform_when_kernels_equal():
+    sh = _shape(n=256, h_q=4, h_kv=1, d=8)
+    p = oracle.params(sh)
+    rng = np.random.default_rng(3)
+    q = _bf16(rng.standard_normal((256, 4, 8)))
+    k = _bf16(np.broadcast_to(rng.standard_normal((1, 1, 8)), (256, 1, 8)))
+    kc1 = oracle.compress_k(p, k)
+    for i in (31, 63, 200, 255):
+        s, _ = oracle.shared_scores_row(p, q, kc1, i, 0)
+        nv = (i - 31) // 16 + 1
+        assert len(s) == nv
+        assert np.allclose(s, 4.0 / nv, rtol=0, atol=1e-14), (i, s)
+
+
+def pin_scores_two_kernels_closed_form():
+    # query 47 sees exactly kernels 0 and 1: S^C1(h) = (sigmoid(-D), sigmoid(D))
+    sh, data = _small_problem(n=64, h_q=4, h_kv=2, d=16, seed=9)
+    p = oracle.params(sh)
+    kc1 = oracle.compress_k(p, data["k"])
+    q, K = _f64(data["q"]), _f64(kc1)
+    for g in range(2):
+        s, _ = oracle.shared_scores_row(p, data["q"], kc1, 47, g)
+        want = np.zeros(2)
+        for hh in range(2):
+            h = g * 2 + hh
+            D = (q[47, h] @ K[1, g] - q[47, h] @ K[0, g]) / np.sqrt(16)
+            want += [1 / (1 + np.exp(D)), 1 / (1 + np.exp(-D))]
+        assert np.allclose(s, want, rtol=1e-13, atol=0), (g, s, want)
+
+
+def pin_scores_torch_softmax():
+    sh, data = _small_problem(n=333, h_q=8, h_kv=2, d=32, seed=21)
+    p = oracle.params(sh)
+    kc1 = oracle.compress_k(p, data["k"])
+    q = torch.from_numpy(_f64(data["q"]))
+    K = torch.from_numpy(_f64(kc1))
+    for i in (40, 100, 332):
+        nv = (i - 31) // 16 + 1
+        for g in range(2):
+            s, lse = oracle.shared_scores_row(p, data["q"], kc1, i, g)
+            z = (q[i, g * 4:(g + 1) * 4] @ K[:nv, g].T) / np.sqrt(32)     # [G, nv]
+            want = torch.softmax(z, dim=-1).sum(0).numpy()
+            assert np.allclose(s, want, rtol=1e-12, atol=1e-15), (i, g)
+            assert np.allclose(lse, torch.logsumexp(z, dim=-1).numpy(), rtol=1e-13, atol=1e-13)
+
+
+def pin_scores_group_mapping():
+    # heads 0,1 form group 0 and heads 2,3 group 1 (consecutive query heads share
+    # a kv head).  Group 0's queries are zero -> uniform scores; group 1's queries
+    # point at kernel 0 of kv head 1 -> concentrated there.
+    sh = _shape(n=128, h_q=4, h_kv=2, d=8)
+    p = oracle.params(sh)
+    k = np.zeros((128, 2, 8), np.float32)
+    k[:32, 1, 0] = 4.0                      # kernel 0 of kv head 1 only
+    q = np.zeros((128, 4, 8), np.float32)
+    q[:, 2:4, 0] = 8.0
+    kb, qb = _bf16(k), _bf16(q)
+    kc1 = oracle.compress_k(p, kb)
+    i = 127
+    nv = (i - 31) // 16 + 1
+    s0, _ = oracle.shared_scores_row(p, qb, kc1, i, 0)
+    s1, _ = oracle.shared_scores_row(p, qb, kc1, i, 1)
+    assert np.allclose(s0, 2.0 / nv, atol=1e-14)
+    # kernel 0 of kv head 1 has mean 4 in dim 0 (tokens 0..31); kernel 1 covers
+    # tokens 16..47 -> mean 2; later kernels 0.  Logits 32/sqrt(8), 16/sqrt(8), 0.
+    z = np.array([32.0, 16.0] + [0.0] * (nv - 2)) / np.sqrt(8)
+    want = 2 * np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+    assert np.allclose(s1, want, rtol=1e-12, atol=1e-15), (s1[:3], want[:3])
+
+
+# --------------------------------------------------------------------------
+# stage 3: max pooling into block scores
+# --------------------------------------------------------------------------
+
+def pin_maxpool_hand():
+    p = oracle.params(_shape())
+    fx = {ln[0]: ln[1:] for ln in _lines("maxpool_hand.txt")}
+    i = int(fx["query"][0])
+    shared = np.array([float(x) for x in fx["shared"]])
+    assert len(shared) == oracle.visible_kernels(p, i)
+    got = oracle.block_scores_row(p, shared, i)
+    assert np.array_equal(got, [float(x) for x in fx["expected"]]), got
+
+
+def pin_maxpool_bruteforce():
+    p = oracle.params(_shape())
+    rng = np.random.default_rng(4)
+    for i in (31, 63, 64, 95, 130, 511, 700):
+        nv = oracle.visible_kernels(p, i)
+        shared = rng.random(nv)
+        got = oracle.block_scores_row(p, shared, i)
+        for b in range(i // 64 + 1):
+            blk = set(range(64 * b, 64 * b + 64))
+            win = [shared[j] for j in range(nv) if blk & set(range(16 * j, 16 * j + 32))]
+            want = max(win) if win else -np.inf
+            assert got[b] == want, (i, b, got[b], want)
+
+
+# --------------------------------------------------------------------------
+# stage 4: selection
+# --------------------------------------------------------------------------
+
+def pin_select_hand():
+    fx = list(_lines("select_hand.txt"))
+    i = int(fx[0][1])
+    cmp_ = np.array([float(x) for x in fx[1][1:]])
+    for ln in fx[2:]:
+        k = int(ln[1])
+        want = [int(x) for x in ln[3:]]
+        p = oracle.params(_shape(k=k, n_init=1, n_local=2))
+        got = oracle.select_row(p, cmp_, i)
+        assert list(got) == want + [-1] * (k - len(want)), (k, got, want)
+
+
+def _select_bruteforce(cmp_, i, k, n_init, n_local, B=64):
+    bi = i // B
+    cand = list(range(bi + 1))
+    if len(cand) <= k:
+        return sorted(cand)
+    forced = [b for b in cand if b < n_init or b > bi - n_local]
+    rest = sorted((b for b in cand if b not in forced), key=lambda b: (-cmp_[b], b))
+    return sorted(forced + rest[:k - len(forced)])
+
+
+def pin_select_bruteforce():
+    rng = np.random.default_rng(8)
+    for trial in range(60):
+        n_init = int(rng.integers(0, 3))
+        n_local = int(rng.integers(1, 3))
+        k = int(rng.integers(n_init + n_local, 20))
+        i = int(rng.integers(0, 64 * 40))
+        # coarse values so that ties are common
+        cmp_ = rng.integers(0, 6, size=i // 64 + 1).astype(np.float64) / 4
+        p = oracle.params(_shape(k=k, n_init=n_init, n_local=n_local))
+        got = [b for b in oracle.select_row(p, cmp_, i) if b >= 0]
+        assert got == _select_bruteforce(cmp_, i, k, n_init, n_local), (trial, got)
+
+
+def pin_select_invariants():
+    sh = synth.CONFIGS["c1"]["shape"]
+    data = synth.make_prefill(sh, seed=0)
+    p = oracle.params(sh)
+    rows = np.array([0, 30, 31, 63, 64, 200, 511, 512, 513, 777, 1500, 2047])
+    out = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows)
+    for r, i in enumerate(rows):
+        bi = i // sh.B
+        sel = out["idx"][r, 0]
+        got = [b for b in sel if b >= 0]
+        assert len(got) == min(sh.k, bi + 1)
+        assert all(x < y for x, y in zip(got, got[1:]))
+        assert all(0 <= b <= bi for b in got)
+        assert all(b == -1 for b in sel[len(got):])
+        forced = {b for b in range(bi + 1) if b < sh.n_init or b > bi - sh.n_local}
+        assert forced <= set(got), (i, got)
+
+
+# --------------------------------------------------------------------------
+# stage 5: attention
+# --------------------------------------------------------------------------
+
+def _sdpa(q, k, v, mask):
+    """torch fp64 attention of q [h_q, d] over keys [T, h_kv, d] with a bool mask [T]."""
+    h_q, d = q.shape
+    G = h_q // k.shape[1]
+    kk = k.repeat_interleave(G, dim=1).permute(1, 0, 2)         # [h_q, T, d]
+    vv = v.repeat_interleave(G, dim=1).permute(1, 0, 2)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q[:, None, :], kk, vv, attn_mask=mask[None, None, :].expand(h_q, 1, -1),
+        scale=1.0 / np.sqrt(d))[:, 0, :]
+    z = (q[:, None, :] * kk).sum(-1) / np.sqrt(d)
+    lse = torch.logsumexp(z.masked_fill(~mask[None, :], -np.inf), dim=-1)
+    return out.numpy(), lse.numpy()
+
+
+def pin_attend_dense_matches_sdpa():
+    # n <= k*B: dense causal attention for every row
+    sh, data = _small_problem(n=150, h_q=4, h_kv=2, d=16, seed=2, k=8)
+    p = oracle.params(sh)
+    rows = np.array([0, 1, 17, 63, 64, 100, 149])
+    out = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows)
+    q, k, v = (torch.from_numpy(_f64(data[x])) for x in ("q", "k", "v"))
+    for r, i in enumerate(rows):
+        mask = torch.arange(150) <= i
+        o, lse = _sdpa(q[i], k, v, mask)
+        assert np.allclose(out["o"][r], o, rtol=1e-12, atol=1e-12), i
+        assert np.allclose(out["lse"][r], lse, rtol=1e-12, atol=1e-12), i
+
+
+def pin_attend_block_mask_matches_sdpa():
+    sh, data = _small_problem(n=700, h_q=4, h_kv=2, d=16, seed=6, k=3)
+    p = oracle.params(sh)
+    rows = np.array([5, 64, 130, 300, 450, 699])
+    out = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows)
+    q, k, v = (torch.from_numpy(_f64(data[x])) for x in ("q", "k", "v"))
+    t = torch.arange(700)
+    for r, i in enumerate(rows):
+        for g in range(2):
+            blocks = [b for b in out["idx"][r, g] if b >= 0]
+            mask = (t <= i) & torch.isin(t // 64, torch.tensor(blocks))
+            o, lse = _sdpa(q[i, 2 * g:2 * g + 2], k[:, g:g + 1], v[:, g:g + 1], mask)
+            assert np.allclose(out["o"][r, 2 * g:2 * g + 2], o, rtol=1e-12, atol=1e-12), (i, g)
+            assert np.allclose(out["lse"][r, 2 * g:2 * g + 2], lse, rtol=1e-12, atol=1e-12)
+
+
+def pin_attend_closed_forms():
+    # equal keys -> uniform weights -> O is the mean of the visible values and
+    # lse = z + log(count)
+    sh = _shape(n=130, h_q=2, h_kv=1, d=8, k=8)
+    p = oracle.params(sh)
+    rng = np.random.default_rng(1)
+    q = _bf16(rng.standard_normal((130, 2, 8)))
+    krow = _bf16(rng.standard_normal(8))
+    k = np.broadcast_to(krow, (130, 1, 8)).copy()
+    v = _bf16(rng.standard_normal((130, 1, 8)))
+    vv = _f64(v)
+    for i in (0, 5, 64, 129):
+        blocks = list(range(i // 64 + 1))
+        o, lse = oracle.attend_row(p, q, k, v, i, 0, blocks)
+        want = vv[:i + 1, 0].mean(0)
+        assert np.allclose(o, want[None], rtol=1e-12, atol=1e-13), i
+        z = _f64(q)[i] @ _f64(krow) / np.sqrt(8)
+        assert np.allclose(lse, z + np.log(i + 1), rtol=1e-12, atol=1e-12)
+
+
+def pin_early_rows_are_dense():
+    # in a sparse sequence, a query with at most k visible blocks attends densely
+    sh, data = _small_problem(n=1000, h_q=2, h_kv=1, d=16, seed=12, k=4)
+    p = oracle.params(sh)
+    rows = np.array([10, 100, 200, 255])
+    out = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows)
+    q, k, v = (torch.from_numpy(_f64(data[x])) for x in ("q", "k", "v"))
+    for r, i in enumerate(rows):
+        o, lse = _sdpa(q[i], k, v, torch.arange(1000) <= i)
+        assert np.allclose(out["o"][r], o, rtol=1e-12, atol=1e-12), i
+
+
+ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]
