@@ -1,0 +1,559 @@
+"""Benchmark of the InfLLM-V2 block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one whole prefill of a 131072-token sequence (h_q=32, h_kv=2,
+d=128, top-k 64 blocks of 64): stage-1 compression, the two-pass scores,
+max-pool + top-k selection and block-sparse attention, through the C ABI
+(infv2_prefill).  Inputs are seeded synthetic bf16 arrays already resident in
+HBM (Q alone is 1.07 GB, larger than L2, so no L2 flush is needed).  Rank 0
+prints one JSON line.  With torchrun, every rank runs its own replica of the
+workload (independent sequences, no collective on the data path) and the
+reported time is the maximum over ranks.
+
+Also reported: a per-stage breakdown timed with CUDA events on the launching
+stream, the roofline of the dominant kernel, an end-to-end figure through host
+buffers, the batched decode step (32 sequences, 16k-128k cached tokens), SM
+clocks sampled during the timed region, and the fp64 CPU oracle timed on a
+bounded sample of query rows.  --impl reference times that oracle as the
+reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from trainable_block_sparse_mean_b200 import synth  # noqa: E402
+
+METRIC = "sparse prefill tokens/s + TFLOP/s at 128k (% of peak); decode µs/token"
+WORKLOAD = "c3: prefill, single sequence n=131072, h_q=32, h_kv=2, d=128, bf16, top-k 64 blocks of 64, 128 needles"
+B, D = 64, 128
+
+
+# ------------------------------------------------------------------ accounting
+
+def visible_kernels(i):
+    i = np.asarray(i, dtype=np.int64)
+    return np.where(i >= 31, (i - 31) // 16 + 1, 0)
+
+
+def prefill_work(shape: synth.Shape, n: int):
+    """Algorithmic FLOPs of one prefill: two score passes over the visible
+    kernels (2*d each per head), attention over the selected visible tokens
+    (4*d per head and key); dense attention over all visible tokens when
+    n <= k*B."""
+    i = np.arange(n, dtype=np.int64)
+    bi = i // B
+    h = shape.h_q
+    if n <= shape.k * B:
+        att_keys = (i + 1).sum()
+        return dict(score=0.0, attn=float(4 * D * h * att_keys), dense=True)
+    score = float(2 * 2 * D * h * visible_kernels(i).sum())
+    sel = np.minimum(shape.k, bi + 1)
+    keys = B * (sel - 1) + (i % B) + 1
+    return dict(score=score, attn=float(4 * D * h * keys.sum()), dense=False)
+
+
+def decode_bytes(shape: synth.Shape, lens):
+    """Algorithmic HBM bytes of one decode step at query positions `lens`:
+    the visible K^C1 rows, the selected K and V rows, q, o and the new K/V."""
+    L = np.asarray(lens, np.int64)
+    bi = L // B
+    sel = np.minimum(shape.k, bi + 1)
+    keys = B * (sel - 1) + (L % B) + 1
+    row = D * 2
+    kc1 = shape.h_kv * visible_kernels(L).sum() * row
+    kv = shape.h_kv * keys.sum() * 2 * row
+    small = len(L) * (2 * shape.h_q * row + 2 * 2 * shape.h_kv * row)
+    return float(kc1 + kv + small)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ peaks / profiles
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per unit from the committed ncu summary, if the kernel's
+    source has not changed since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank, dist):
+    import torch
+    from trainable_block_sparse_mean_b200 import infv2
+    from trainable_block_sparse_mean_b200.workloads import DecodeState, to_dev
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shape = synth.CONFIGS["c3"]["shape"]
+    n = shape.n
+    p = infv2.params_of(shape)
+    data = synth.make_prefill(shape, seed=rank)
+    q, k, v = to_dev(data["q"], dev), to_dev(data["k"], dev), to_dev(data["v"], dev)
+    cu = [0, n]
+    ws = torch.empty(infv2.infv2_prefill_workspace_size(p, cu), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.h_q, n), device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def step():
+        infv2.infv2_prefill(p, q, k, v, cu, workspace=ws, o=o, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if infv2.infv2_device_status() != 0:
+        raise RuntimeError("kernel error word set during warm-up")
+
+    clocks = ClockSampler(local_rank).start() if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(ms)
+    pl = infv2.infv2_prefill_workspace_size(p, cu)
+    chunk_rows = _chunk_rows(p, n)
+    n_chunks = (n + chunk_rows - 1) // chunk_rows
+    launches_per_step = 1 + 2 * n_chunks + 1
+
+    # ---- per-stage breakdown on the same stream (CUDA events between launches)
+    stage = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows)
+    # ---- end to end through host buffers
+    e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks)
+    # ---- decode
+    dec = _decode(args, infv2, torch, shape, rank, dev, stream, max_over_ranks, DecodeState)
+    if infv2.infv2_device_status() != 0:
+        raise RuntimeError("kernel error word set during the benchmark")
+
+    work = prefill_work(shape, n)
+    flops = work["score"] + work["attn"]
+    peaks = measured_peaks()
+    tps = world * n / (ms / 1e3)
+    tflops = world * flops / (ms / 1e3) / 1e12
+    # dominant kernel and its roofline
+    dom = max(stage["per_kernel"], key=lambda kk: stage["per_kernel"][kk]["ms_per_step"])
+    dk = stage["per_kernel"][dom]
+    unit_flops = {"score_kernel": work["score"], "sparse_attn_kernel": work["attn"],
+                  "select_kernel": None, "compress_k_kernel": None}[dom]
+    if unit_flops is not None:
+        per_launch = unit_flops / dk["launches_per_step"]
+        achieved = per_launch / (dk["ms_per_launch"] / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": peaks["source"] + " burst bf16 (cuBLAS)"}
+    else:
+        byts = dk.get("bytes_per_step", 0.0) / dk["launches_per_step"]
+        achieved = byts / (dk["ms_per_launch"] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peaks["source"]}
+    tr = recorded_traffic(dom)
+    roof["traffic"] = (tr["dram_bytes_per_launch_per_token"] * n / dk["launches_per_step"]
+                       if tr and "dram_bytes_per_launch_per_token" in tr else
+                       (tr["dram_bytes_per_launch"] if tr and "dram_bytes_per_launch" in tr else None))
+    sel_ms = sum(stage["per_kernel"][x]["ms_per_step"] for x in
+                 ("compress_k_kernel", "score_kernel", "select_kernel"))
+    out = {
+        "metric": METRIC, "value": round(tps, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/V, K with per-block offsets and 128 planted needles)",
+        "config": {"workload": WORKLOAD, "n": n, "h_q": shape.h_q, "h_kv": shape.h_kv,
+                   "d": shape.d, "block": shape.B, "top_k_blocks": shape.k,
+                   "n_init": shape.n_init, "n_local": shape.n_local, "l_c1": shape.l_c1,
+                   "s_c1": shape.s_c1, "pool_l": shape.pool_l, "pool_s": shape.pool_s,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "no flush: Q (1.07 GB) alone exceeds the 126 MB L2"},
+        "tflops": round(tflops, 2),
+        "tflops_frac_of_peak": round(tflops / world / peaks["bf16_tflops"], 4),
+        "algorithmic_tflop_per_step": {"score": round(work["score"] / 1e12, 3),
+                                       "attention": round(work["attn"] / 1e12, 3)},
+        "selection_share": round(sel_ms / stage["ms_per_step"], 4),
+        "stages": stage["per_kernel"],
+        "roofline": roof,
+        "e2e": e2e,
+        "decode": dec,
+        "gpu_launches": launches_per_step * args.steps,
+        "peaks": peaks,
+    }
+    if clk:
+        out["clocks"] = clk
+    return out
+
+
+def _chunk_rows(p, n):
+    # mirrors the library's chunking of S^shared (256 MiB budget, multiples of 128 rows)
+    ld = ((max((n - 32) // 16 + 1, 4 * ((n + 63) // 64)) + 31) // 32) * 32
+    rows = (256 << 20) // (p.h_kv * ld * 4)
+    rows = max(128, (rows // 128) * 128)
+    return min(rows, n)
+
+
+def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows):
+    """Run the prefill stage by stage through the C ABI, with CUDA events
+    around every launch, and average each kernel's duration."""
+    n = shape.n
+    nc = infv2.num_kernels(p, n)
+    ld = infv2.shared_ld(n)
+    kc1 = ws[: nc * p.h_kv * 128 * 2].view(torch.bfloat16).view(nc, p.h_kv, 128)
+    off_sh = ((nc * p.h_kv * 256) + 255) // 256 * 256
+    s_sh = ws[off_sh: off_sh + p.h_kv * chunk_rows * ld * 4].view(torch.float32).view(p.h_kv, chunk_rows, ld)
+    idx = torch.empty((p.h_kv, n, p.k), dtype=torch.int32, device=q.device)
+    names = ["compress_k_kernel", "score_kernel", "select_kernel", "sparse_attn_kernel"]
+
+    def one(record):
+        evs = []
+        def ev():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            return e
+        a = ev()
+        infv2.infv2_compress_k(p, k, kc1)
+        evs.append(("compress_k_kernel", a, ev()))
+        for q0 in range(0, n, chunk_rows):
+            ql = min(chunk_rows, n - q0)
+            a = ev()
+            infv2.infv2_block_scores(p, q, kc1, n, q0, ql, s_sh[:, :ql] if ql == chunk_rows else
+                                     s_sh.view(-1)[: p.h_kv * ql * ld].view(p.h_kv, ql, ld), ld)
+            b = ev()
+            infv2.infv2_select_topk(p, s_sh.view(-1)[: p.h_kv * ql * ld].view(p.h_kv, ql, ld), ld, n,
+                                    q0, ql, idx)
+            evs.append(("score_kernel", a, b))
+            evs.append(("select_kernel", b, ev()))
+        a = ev()
+        infv2.infv2_sparse_attn(p, q, k, v, idx, o, lse)
+        evs.append(("sparse_attn_kernel", a, ev()))
+        return evs
+
+    for _ in range(max(1, args.warmup)):
+        one(False)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    all_evs = []
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        all_evs.append(one(True))
+    e1.record(stream)
+    torch.cuda.synchronize()
+    per = {nm: {"ms_per_step": 0.0, "launches_per_step": 0} for nm in names}
+    for evs in all_evs:
+        for nm, a, b in evs:
+            per[nm]["ms_per_step"] += a.elapsed_time(b)
+            per[nm]["launches_per_step"] += 1
+    for nm in names:
+        per[nm]["ms_per_step"] /= steps
+        per[nm]["launches_per_step"] //= steps
+        per[nm]["ms_per_launch"] = per[nm]["ms_per_step"] / max(1, per[nm]["launches_per_step"])
+    # algorithmic bytes of the memory-bound stages
+    per["compress_k_kernel"]["bytes_per_step"] = float(n * p.h_kv * 256 + nc * p.h_kv * 256)
+    vis = visible_kernels(np.arange(n)).sum()
+    per["select_kernel"]["bytes_per_step"] = float(p.h_kv * vis * 4 + p.h_kv * n * p.k * 4)
+    for nm in names:
+        per[nm] = {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in per[nm].items()}
+    return dict(per_kernel=per, ms_per_step=e0.elapsed_time(e1) / steps)
+
+
+def _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks):
+    """Same metric through the C ABI with host buffers: every step copies the
+    inputs from pinned host memory and reads the output back."""
+    from trainable_block_sparse_mean_b200.workloads import to_dev
+    qh = torch.from_numpy(data["q"].view(np.int16)).pin_memory()
+    kh = torch.from_numpy(data["k"].view(np.int16)).pin_memory()
+    vh = torch.from_numpy(data["v"].view(np.int16)).pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    qd = torch.empty(qh.shape, dtype=torch.int16, device=dev)
+    kd = torch.empty(kh.shape, dtype=torch.int16, device=dev)
+    vd = torch.empty(vh.shape, dtype=torch.int16, device=dev)
+    od = torch.empty(qh.shape, dtype=torch.int16, device=dev)
+
+    def step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        infv2.infv2_prefill(p, qd.view(torch.bfloat16), kd.view(torch.bfloat16),
+                            vd.view(torch.bfloat16), cu, workspace=ws, o=od.view(torch.bfloat16))
+        oh.copy_(od, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps)
+    h2d = qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2
+    d2h = oh.numel() * 2
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": round(world * shape.n / (ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, DecodeState):
+    cfg = synth.CONFIGS["c4"]
+    sh = cfg["shape"]
+    steps_avail = cfg["steps"]
+    data = synth.make_decode(sh, cfg["batch"], cfg["len_lo"], cfg["len_hi"], steps_avail,
+                             seed=rank)
+    st = DecodeState(sh, data, device=dev)
+    o = torch.empty((cfg["batch"], sh.h_q, sh.d), dtype=torch.bfloat16, device=dev)
+    warm = min(args.warmup, 8)
+    for t in range(warm):
+        st.step(t, o=o)
+    torch.cuda.synchronize()
+    timed = min(steps_avail - warm, 48)
+    evs = []
+    for t in range(warm, warm + timed):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st.step(t, o=o)
+        b.record(stream)
+        evs.append((a, b, t))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b, _ in evs]
+    us = max_over_ranks(float(np.median(times)) * 1e3)
+    lens_mid = data["lens"] + warm + timed // 2
+    byts = decode_bytes(sh, lens_mid)
+    peaks = measured_peaks()
+    gbs = byts / (us / 1e6) / 1e9
+    return {"workload": "c4: batch 32, one query token each, cache lengths U[16384, 131072] (seed-0 mean %.0f), h_q=32, h_kv=2, top-k 64" % data["lens"].mean(),
+            "us_per_step": round(us, 2), "us_per_token_per_sequence": round(us, 2),
+            "us_per_token_aggregate": round(us / cfg["batch"], 3),
+            "launches_per_step": 7, "algorithmic_bytes_per_step": int(byts),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(target_s=12.0, seed=0):
+    """Time the fp64 oracle on a bounded random sample of query rows of the
+    128k workload (rows drawn uniformly; cost grows with the row index)."""
+    import oracle
+    shape = synth.CONFIGS["c3"]["shape"]
+    data = synth.make_prefill(shape, seed=0)
+    op = oracle.params(shape)
+    rng = np.random.default_rng(seed)
+    threads = oracle.num_threads()
+    # calibrate on one batch of `threads` rows, then size the sample
+    rows = rng.integers(0, shape.n, size=threads).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(op, data["q"], data["k"], data["v"], rows)
+    t_cal = time.perf_counter() - t0
+    n_rows = max(threads, int(threads * target_s / max(t_cal, 1e-3)))
+    rows = rng.integers(0, shape.n, size=n_rows).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(op, data["q"], data["k"], data["v"], rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(n_rows / dt, 3), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "%d query rows drawn uniformly from the 131072-token sequence (all stages, "
+                      "fp64, OpenMP over rows), %.1f s" % (n_rows, dt)}, data, shape
+
+
+def run_reference(args):
+    import oracle
+    oracle.build()
+    shape = synth.CONFIGS["c3"]["shape"]
+    data = synth.make_prefill(shape, seed=0)
+    op = oracle.params(shape)
+    threads = oracle.num_threads()
+    rng = np.random.default_rng(1)
+    rows = rng.integers(0, shape.n, size=threads).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(op, data["q"], data["k"], data["v"], rows)
+    per_batch = time.perf_counter() - t0
+    # size each step to about 6 s of CPU work
+    rows_per_step = max(threads, int(threads * 6.0 / max(per_batch, 1e-3)))
+    for _ in range(args.warmup):
+        r = rng.integers(0, shape.n, size=threads).astype(np.int32)
+        oracle.prefill_rows(op, data["q"], data["k"], data["v"], r)
+    t_total, n_total = 0.0, 0
+    for _ in range(args.steps):
+        r = rng.integers(0, shape.n, size=rows_per_step).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(op, data["q"], data["k"], data["v"], r)
+        t_total += time.perf_counter() - t0
+        n_total += rows_per_step
+    v = n_total / t_total
+    sample = ("%d query rows per step drawn uniformly from the 131072-token sequence "
+              "(all stages, fp64, OpenMP over rows)" % rows_per_step)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * t_total / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)))
+        return 0
+
+    from trainable_block_sparse_mean_b200 import build as lib_build
+    if rank == 0 or world == 1:
+        lib_build.build()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+        dist.barrier()
+    try:
+        out = run_ours(args, rank, world, local_rank, dist)
+        if rank == 0 and not args.no_cpu_baseline:
+            cpu, _, _ = oracle_sample()
+            out["cpu_baseline"] = cpu
+        if rank == 0:
+            print(json.dumps(out))
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,202 @@
+/*
+ * infv2.h -- C ABI of libinfv2.so: InfLLM-V2 dense-sparse switchable attention
+ * for one causal GQA layer, hand-written for NVIDIA B200 (sm_100a).
+ *
+ * Method (the InfLLM-V2 paper, arXiv 2509.24663, and its public summaries):
+ *   1. stage-1 compression: K^C1 = mean of K over kernels of l_C1 = B/2 tokens
+ *      with stride s_C1 = B/4 (paper notes, key design 3; MiniCPM4 blog,
+ *      semantic kernels);
+ *   2. S^C1 = softmax(Q K^C1^T) over the causally visible kernels and the GQA
+ *      group sum S^shared = sum_h S^C1(h), computed in two passes (log-sum-exp,
+ *      then normalise-and-sum) so that only S^shared reaches memory (paper
+ *      notes, key design 4; arXiv summary, section 3 "Efficient Implementation");
+ *   3. block scores S^cmp = max pooling of S^shared over the kernels that
+ *      intersect each block (l = 5, s = 4) (paper notes, key design 3; MiniCPM4
+ *      blog, semantic kernels);
+ *   4. selection I(i) = I_init u I_local(i) u top-k(S^cmp), one set per query
+ *      token and kv head (paper notes, key design 2; MiniCPM4 blog, top-k
+ *      sharing);
+ *   5. block-sparse causal attention over the selected blocks, returning O and
+ *      the log-sum-exp (arXiv summary, Appendix A), or dense causal attention
+ *      when the sequence has at most k blocks (MiniCPM4 blog, semantic kernels).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, unless a
+ *     parameter says "host".  The library allocates no memory; scratch space
+ *     is the caller's `workspace`.
+ *   - bf16 tensors are raw 16-bit patterns (e.g. torch.bfloat16 storage);
+ *     every tensor is dense, row-major, 16-byte aligned.
+ *   - Token layout ("thd"): q [n, h_q, d], k and v [n, h_kv, d]; query head h
+ *     belongs to kv head h / (h_q / h_kv).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return an infv2_status for argument / launch errors.  Errors
+ *     detected inside a kernel (a bounded wait that timed out) are recorded in
+ *     a per-device word read by infv2_device_status().
+ *   - No call retains a pointer after it returns; calls that share output or
+ *     workspace memory must be ordered on the caller's streams.
+ */
+#ifndef INFV2_H
+#define INFV2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* infv2_stream_t;
+
+enum infv2_status {
+  INFV2_OK = 0,
+  INFV2_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shape */
+  INFV2_ERR_UNSUPPORTED = 2, /* valid for the method but not for this build's kernels */
+  INFV2_ERR_WORKSPACE = 3,   /* workspace smaller than the *_workspace_size answer */
+  INFV2_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  INFV2_ERR_TIMEOUT = 5      /* a kernel's bounded wait ran out (device word only) */
+};
+
+/* Method parameters.
+ *   B        block size in tokens (selection and attention granularity)
+ *   l_c1     stage-1 kernel length (B/2 in the paper)
+ *   s_c1     stage-1 kernel stride (B/4 in the paper)
+ *   pool_l   max-pool length in kernels (5): kernels intersecting a block
+ *   pool_s   max-pool stride in kernels (4)
+ *   n_init   initial blocks always selected
+ *   n_local  local blocks always selected: {b_i - n_local + 1 .. b_i}
+ *   k        total blocks selected per query, init and local included
+ *   h_q, h_kv, d   query heads, kv heads, head dim
+ *   scale    logit scale of both the scores and the attention (1/sqrt(d))
+ *   window   sliding window (tokens) that the local blocks must cover:
+ *            n_local >= ceil(window / B) + 1 is enforced (0 = no window)
+ * This build's kernels support d = 128, B = 64, l_c1 = 32, s_c1 = 16,
+ * pool_l = 5, pool_s = 4, h_q % h_kv == 0 with G = h_q/h_kv in {1,2,4,8,16},
+ * k >= n_init + n_local, n_local >= 1 and k <= 256.  Other values return
+ * INFV2_ERR_UNSUPPORTED. */
+typedef struct infv2_params {
+  int B, l_c1, s_c1, pool_l, pool_s;
+  int n_init, n_local, k;
+  int h_q, h_kv, d;
+  float scale;
+  int window;
+} infv2_params;
+
+/* Fill *p with the paper's hyper-parameters (B=64, l_c1=32, s_c1=16, l=5,
+ * s=4, n_init=1, n_local=2, k=64, d=128, scale=1/sqrt(128)) for h_q, h_kv. */
+void infv2_default_params(infv2_params* p, int h_q, int h_kv);
+
+/* Validate *p against the method and this build.  Returns INFV2_OK,
+ * INFV2_ERR_INVALID_ARG or INFV2_ERR_UNSUPPORTED. */
+int infv2_check_params(const infv2_params* p);
+
+/* Static text for a status code (never NULL). */
+const char* infv2_status_string(int status);
+
+/* Number of complete stage-1 kernels of an n-token sequence:
+ * n >= l_c1 ? (n - l_c1) / s_c1 + 1 : 0. */
+int infv2_num_kernels(const infv2_params* p, int n);
+
+/* Read and clear this device's kernel error word (waits for `stream`).
+ * Returns INFV2_OK, INFV2_ERR_TIMEOUT, or INFV2_ERR_CUDA if the read fails. */
+int infv2_device_status(infv2_stream_t stream);
+
+/* Stage 1 (paper notes, key design 3): K^C1[j, g, :] = bf16 round-to-nearest-
+ * even of the exact mean of K[t, g, :] over t = j*s_c1 .. j*s_c1 + l_c1 - 1.
+ *   k    bf16 [n, h_kv, d]            (input)
+ *   kc1  bf16 [num_kernels(n), h_kv, d] (output)
+ * n = 0 or n < l_c1 writes nothing. */
+int infv2_compress_k(const infv2_params* p, const void* k, int n, void* kc1,
+                     infv2_stream_t stream);
+
+/* Stage 2, fused two-pass scores (paper notes, key design 4; arXiv summary,
+ * section 3): for query rows i in [q_begin, q_begin + q_len) of an n-token
+ * sequence and kv head g, with J(i) the kernels j where j*s_c1 + l_c1 - 1 <= i,
+ *   S^shared[g, i - q_begin, j] = sum_{h in group g} exp(z_hj - lse_h),
+ *   z_hj = scale * q[i, h, :] . kc1[j, g, :],  lse_h = log sum_{j in J(i)} exp(z_hj).
+ *   q         bf16 [n, h_q, d];  kc1  bf16 [num_kernels(n), h_kv, d]
+ *   s_shared  fp32 [h_kv, q_len, ld] (output); only j < |J(i)| is written
+ *   ld        row pitch in floats, >= num_kernels(n), multiple of 4
+ *   score_lse fp32 [h_q, q_len] (output, nullable): lse_h (natural log),
+ *             -inf for rows with no visible kernel. */
+int infv2_block_scores(const infv2_params* p, const void* q, const void* kc1, int n, int q_begin,
+                       int q_len, float* s_shared, int ld, float* score_lse,
+                       infv2_stream_t stream);
+
+/* Stages 3-4 (paper notes, key designs 2-3; MiniCPM4 blog, semantic kernels):
+ * for each row i in [q_begin, q_begin + q_len) and kv head g, block scores
+ *   S^cmp[b] = max over visible kernels j intersecting block b of S^shared[j],
+ * then I(i) = all of 0..i/B when that is at most k blocks, else the init and
+ * local blocks plus the highest-scoring others up to k in total (equal scores:
+ * lower block first).
+ *   s_shared  fp32 [h_kv, q_len, ld] as written by infv2_block_scores
+ *   idx       int32 [h_kv, n, k] (output): rows q_begin.. written, ascending,
+ *             padded with -1. */
+int infv2_select_topk(const infv2_params* p, const float* s_shared, int ld, int n, int q_begin,
+                      int q_len, int* idx, infv2_stream_t stream);
+
+/* Stage 5, block-sparse attention (arXiv summary, Appendix A): for every
+ * query i and head h of group g, softmax attention over the tokens t <= i of
+ * the blocks listed in idx[g, i, :] (entries < 0 ignored).
+ *   q bf16 [n, h_q, d]; k, v bf16 [n, h_kv, d]; idx int32 [h_kv, n, k]
+ *   o   bf16 [n, h_q, d] (output)
+ *   lse fp32 [h_q, n] (output, nullable): natural log-sum-exp of the logits. */
+int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const void* v,
+                      const int* idx, int n, void* o, float* lse, infv2_stream_t stream);
+
+/* Dense causal attention with the same weights (MiniCPM4 blog: sequences of
+ * at most k blocks switch to dense attention).  Layouts as infv2_sparse_attn. */
+int infv2_dense_attn(const infv2_params* p, const void* q, const void* k, const void* v, int n,
+                     void* o, float* lse, infv2_stream_t stream);
+
+/* Workspace bytes that infv2_prefill needs for this varlen batch.
+ *   cu_seqlens_host  HOST int32 [batch + 1], cu_seqlens_host[0] = 0. */
+int infv2_prefill_workspace_size(const infv2_params* p, const int* cu_seqlens_host, int batch,
+                                 size_t* bytes);
+
+/* The whole layer over a packed varlen batch (paper notes, overall framework:
+ * dense for short sequences, sparse for long ones).  Sequence s owns tokens
+ * cu_seqlens_host[s] .. cu_seqlens_host[s+1]-1 of q [T, h_q, d], k/v
+ * [T, h_kv, d]; it takes dense attention if its length n <= k*B, else stages
+ * 1-5.  Outputs: o bf16 [T, h_q, d]; lse fp32 [h_q, T] (nullable); idx_out
+ * int32 [h_kv, T, k] (nullable; rows of dense sequences are not written).
+ * workspace: device scratch of at least infv2_prefill_workspace_size bytes,
+ * 256-byte aligned. */
+int infv2_prefill(const infv2_params* p, const void* q, const void* k, const void* v,
+                  const int* cu_seqlens_host, int batch, void* workspace, size_t ws_bytes,
+                  int* idx_out, void* o, float* lse, infv2_stream_t stream);
+
+/* Workspace bytes that infv2_decode needs. */
+int infv2_decode_workspace_size(const infv2_params* p, int batch, int cap, size_t* bytes);
+
+/* One decode step for a batch of sequences, each with its own KV cache
+ * (MiniCPM4 blog, query/key granularity: one query token selects its own
+ * blocks, which is what makes decoding fast).  For sequence s with L =
+ * seqlens[s] cached tokens (0 <= L < cap), the step
+ *   1. writes k_new[s], v_new[s] to cache position L and, when that token
+ *      completes a stage-1 kernel (L + 1 >= l_c1 and (L + 1 - l_c1) % s_c1
+ *      == 0), writes K^C1 of kernel (L + 1 - l_c1) / s_c1 to kc1_cache;
+ *   2. computes S^shared, S^cmp and I(L) for the query at position L;
+ *   3. attends over the selected tokens (dense when L + 1 <= k*B);
+ *   4. increments seqlens[s].
+ *   q        bf16 [batch, h_q, d];  k_new, v_new bf16 [batch, h_kv, d]
+ *   k_cache, v_cache  bf16 [batch, h_kv, cap, d]
+ *   kc1_cache         bf16 [batch, h_kv, num_kernels(cap), d]
+ *   seqlens  int32 [batch] (device, read and incremented)
+ *   o        bf16 [batch, h_q, d];  lse fp32 [batch, h_q] (nullable)
+ *   idx_out  int32 [batch, h_kv, k] (nullable) */
+int infv2_decode(const infv2_params* p, const void* q, const void* k_new, const void* v_new,
+                 void* k_cache, void* v_cache, void* kc1_cache, int* seqlens, int batch, int cap,
+                 void* workspace, size_t ws_bytes, int* idx_out, void* o, float* lse,
+                 infv2_stream_t stream);
+
+/* Self-test of the bounded-wait error path: launches one kernel that waits
+ * on a barrier nobody arrives at, with the given limit in microseconds; the
+ * kernel gives up, records INFV2_ERR_TIMEOUT and exits normally.  Read the
+ * result with infv2_device_status(). */
+int infv2_selftest_timeout(int limit_us, infv2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFV2_H */

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function declared in include/infv2.h, and its host-only logic
+(parameter validation, sizes, argument errors) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from trainable_block_sparse_mean_b200 import build as build_mod
+from trainable_block_sparse_mean_b200 import infv2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "infv2.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build_mod.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(infv2_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert set(declared_functions()) == set(infv2.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(infv2.LIB_PATH)
+    missing = [s for s in declared_functions() if not hasattr(lib, s)]
+    assert not missing, missing
+
+
+def test_default_params_and_checks():
+    p = infv2.params(32, 2)
+    assert (p.B, p.l_c1, p.s_c1, p.pool_l, p.pool_s, p.d, p.k) == (64, 32, 16, 5, 4, 128, 64)
+    assert abs(p.scale - 128 ** -0.5) < 1e-7
+    assert infv2.infv2_check_params(p) == infv2.OK
+    bad = infv2.params(32, 2)
+    bad.h_q = 30  # not a multiple of h_kv... 30 % 2 == 0 but G = 15 unsupported
+    assert infv2.infv2_check_params(bad) == infv2.ERR_UNSUPPORTED
+    bad = infv2.params(32, 3)
+    assert infv2.infv2_check_params(bad) == infv2.ERR_INVALID_ARG
+    bad = infv2.params(32, 2, k=2, n_init=1, n_local=2)   # k < n_init + n_local
+    assert infv2.infv2_check_params(bad) == infv2.ERR_INVALID_ARG
+    bad = infv2.params(32, 2, window=200, n_local=2)      # needs n_local >= ceil(200/64)+1 = 5
+    assert infv2.infv2_check_params(bad) == infv2.ERR_INVALID_ARG
+    ok = infv2.params(32, 2, window=200, n_local=5)
+    assert infv2.infv2_check_params(ok) == infv2.OK
+    bad = infv2.params(32, 2)
+    bad.d = 64
+    assert infv2.infv2_check_params(bad) == infv2.ERR_UNSUPPORTED
+    bad = infv2.params(32, 2)
+    bad.n_local = 0
+    assert infv2.infv2_check_params(bad) == infv2.ERR_INVALID_ARG
+    assert infv2.infv2_check_params(infv2.params(64, 2)) == infv2.ERR_UNSUPPORTED  # G = 32
+
+
+def test_num_kernels_matches_definition():
+    p = infv2.params(4, 1)
+    for n in range(0, 300):
+        want = (n - 32) // 16 + 1 if n >= 32 else 0
+        assert infv2.num_kernels(p, n) == want
+
+
+def test_status_strings():
+    for st in range(6):
+        assert infv2.status_string(st)
+    assert infv2.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes_are_host_only():
+    p = infv2.params(32, 2)
+    # all-dense batch needs no workspace
+    assert infv2.infv2_prefill_workspace_size(p, [0, 1024, 3072]) == 0
+    n = 131072
+    ws = infv2.infv2_prefill_workspace_size(p, [0, n])
+    nc = (n - 32) // 16 + 1
+    assert ws >= nc * 2 * 128 * 2 + 2 * n * 64 * 4
+    assert infv2.infv2_decode_workspace_size(p, 32, 131136) > 0
+    with pytest.raises(infv2.Infv2Error):
+        infv2.infv2_prefill_workspace_size(p, [5, 100])   # cu_seqlens[0] must be 0
+    with pytest.raises(infv2.Infv2Error):
+        infv2.infv2_prefill_workspace_size(p, [0, 100, 50])  # negative length
+
+
+def test_argument_errors_before_any_launch():
+    L = infv2.lib()
+    p = infv2.params(32, 2)
+    P = ctypes.byref(p)
+    assert L.infv2_compress_k(P, None, 100, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_compress_k(P, None, -1, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_compress_k(P, None, 0, None, None) == infv2.OK       # nothing to do
+    assert L.infv2_block_scores(P, None, None, 100, 50, 60, None, 128, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_select_topk(P, None, 128, 100, 0, 0, None, None) == infv2.OK
+    assert L.infv2_select_topk(P, None, 6, 100, 0, 10, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_sparse_attn(P, None, None, None, None, 10, None, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_dense_attn(P, None, None, None, 0, None, None, None) == infv2.OK
+    assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,
+                          None, None) == infv2.OK
+    assert L.infv2_selftest_timeout(0, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_check_params(None) == infv2.ERR_INVALID_ARG

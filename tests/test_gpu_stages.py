@@ -1,0 +1,186 @@
+"""Per-stage parity of the CUDA library against the fp64 oracle (small sizes
+that still span several tiles and a ragged tail)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from trainable_block_sparse_mean_b200 import build as build_mod
+from trainable_block_sparse_mean_b200 import infv2, synth
+from trainable_block_sparse_mean_b200.workloads import to_dev, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build_mod.build()
+    infv2.lib()
+
+
+def _problem(n, h_q, h_kv, k=8, seed=0, n_needles=0):
+    sh = synth.Shape(n=n, h_q=h_q, h_kv=h_kv, k=k, n_needles=n_needles)
+    return sh, synth.make_prefill(sh, seed=seed)
+
+
+def _sample_rows(n, count, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [r for r in (0, 1, 30, 31, 32, 46, 47, 63, 64, 127, 128, 511, 512, n - 2, n - 1) if 0 <= r < n]
+    extra = rng.integers(0, n, size=count) if n > 0 else []
+    return np.unique(np.array(fixed + list(extra), dtype=np.int64)).astype(np.int32)
+
+
+# ---------------------------------------------------------------- stage 1
+
+@pytest.mark.parametrize("n,h_kv", [(2048, 1), (1000, 2), (31, 2), (32, 1), (47, 2), (4177, 2)])
+def test_compress_bit_exact(n, h_kv):
+    sh, d = _problem(n, 2 * h_kv, h_kv)
+    p = infv2.params_of(sh)
+    kc1 = infv2.infv2_compress_k(p, to_dev(d["k"]))
+    torch.cuda.synchronize()
+    want = oracle.compress_k(oracle.params(sh), d["k"])
+    got = to_host_bits(kc1) if kc1.numel() else np.zeros((0, h_kv, 128), np.uint16)
+    assert got.shape == want.shape
+    assert np.array_equal(got, want)
+
+
+def test_compress_extreme_values_bit_exact():
+    # wide magnitude spread, ties and signed zeros inside kernels
+    sh = synth.Shape(n=256, h_q=2, h_kv=2)
+    rng = np.random.default_rng(5)
+    k = (rng.standard_normal((256, 2, 128)) * np.exp(rng.uniform(-20, 20, (256, 2, 128)))).astype(np.float32)
+    k[:40, 0, :8] = 1.0
+    k[7, 0, :8] = np.array([1.125, 1.375, 1.25, 1.75, 2.0, 1.0625, 1.1875, -0.0], np.float32)
+    kb = synth.bf16_bits(k)
+    p = infv2.params_of(sh)
+    got = to_host_bits(infv2.infv2_compress_k(p, to_dev(kb)))
+    want = oracle.compress_k(oracle.params(sh), kb)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- stage 2
+
+SCORE_REL = 2e-5   # fp32 tensor-core dot products + fp32 softmax vs fp64
+
+
+@pytest.mark.parametrize("n,h_q,h_kv,q_begin,q_len", [
+    (2048, 4, 1, 0, 2048),        # c1 shape, G=4 (32 tokens per tile)
+    (3000, 32, 2, 0, 3000),       # G=16, ragged tail, 188 kernels (2 tiles)
+    (3000, 32, 2, 1000, 1333),    # a chunk in the middle of the sequence
+    (700, 8, 1, 0, 700),          # G=8
+    (600, 2, 2, 0, 600),          # G=1 (128 tokens per tile)
+    (900, 4, 2, 0, 900),          # G=2
+])
+def test_block_scores_match_oracle(n, h_q, h_kv, q_begin, q_len):
+    sh, d = _problem(n, h_q, h_kv, seed=n + h_q)
+    p = infv2.params_of(sh)
+    op = oracle.params(sh)
+    kc1 = infv2.infv2_compress_k(p, to_dev(d["k"]))
+    ld = infv2.shared_ld(n)
+    slse = torch.full((h_q, q_len), 7.0, device="cuda")
+    s = infv2.infv2_block_scores(p, to_dev(d["q"]), kc1, n, q_begin, q_len, ld=ld, score_lse=slse)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    s = s.cpu().numpy()
+    slse = slse.cpu().numpy()
+    rows = _sample_rows(n, 40, seed=n)
+    rows = rows[(rows >= q_begin) & (rows < q_begin + q_len)]
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows, want_shared=True, want_score_lse=True)
+    for r, i in enumerate(rows):
+        nv = oracle.visible_kernels(op, i)
+        for g in range(h_kv):
+            want = ref["shared"][r, g, :nv]
+            got = s[g, i - q_begin, :nv]
+            err = np.abs(got - want) / np.maximum(np.abs(want), 1e-30)
+            assert err.max(initial=0) <= SCORE_REL, (i, g, err.max(), int(err.argmax()))
+        lw = ref["score_lse"][r]
+        lg = slse[:, i - q_begin]
+        if nv == 0:
+            assert np.all(np.isneginf(lg))
+        else:
+            assert np.allclose(lg, lw, rtol=0, atol=2e-5), (i, lg - lw)
+
+
+# ---------------------------------------------------------------- stages 3-4
+
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64)])
+def test_select_exact_on_oracle_scores(n, h_q, h_kv, k):
+    """The selection decision is taken on the same fp32 values on both sides."""
+    sh, d = _problem(n, h_q, h_kv, k=k, seed=3)
+    op = oracle.params(sh)
+    p = infv2.params_of(sh)
+    rows = _sample_rows(n, 200, seed=1)
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows, want_shared=True)
+    sh32 = ref["shared"].astype(np.float32)          # [rows, h_kv, nc]
+    nc = sh32.shape[2]
+    # quantise a copy to create exact ties in the block scores
+    ties = np.round(sh32 * 64) / 64
+    for vals in (sh32, ties):
+        ld = infv2.shared_ld(n)
+        buf = np.zeros((h_kv, len(rows), ld), np.float32)
+        buf[:, :, :nc] = vals.transpose(1, 0, 2)
+        # the GPU select reads the row of query i at position (i - q_begin); give
+        # each sampled row its own one-row call
+        got = np.zeros((len(rows), h_kv, k), np.int32)
+        dev = torch.from_numpy(buf).cuda()
+        idx = torch.full((h_kv, n, k), -2, dtype=torch.int32, device="cuda")
+        for r, i in enumerate(rows):
+            row = dev[:, r:r + 1, :].contiguous()
+            infv2.infv2_select_topk(p, row, ld, n, int(i), 1, idx)
+        torch.cuda.synchronize()
+        idx = idx.cpu().numpy()
+        for r, i in enumerate(rows):
+            got[r] = idx[:, i, :]
+        want, _ = oracle.select_rows(op, vals.astype(np.float64), rows, (n + 63) // 64)
+        assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- stage 5
+
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (3001, 32, 2, 16), (1500, 16, 2, 4)])
+def test_sparse_attn_on_oracle_indices(n, h_q, h_kv, k):
+    sh, d = _problem(n, h_q, h_kv, k=k, seed=11)
+    op = oracle.params(sh)
+    p = infv2.params_of(sh)
+    rows = np.arange(n, dtype=np.int32) if n <= 2048 else _sample_rows(n, 150)
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows)
+    idx = np.full((h_kv, n, k), -1, np.int32)
+    idx[:, :, 0] = (np.arange(n) // 64)[None, :]   # rows not sampled: own block only
+    idx[:, rows, :] = ref["idx"].transpose(1, 0, 2)
+    lse = torch.empty((h_q, n), device="cuda")
+    o = infv2.infv2_sparse_attn(p, to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]),
+                                torch.from_numpy(idx).cuda(), lse=lse)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    og = synth.bf16_to_f32(to_host_bits(o))[rows]
+    parity.assert_outputs_close(og, ref["o"], "sparse_attn")
+    lg = lse.cpu().numpy()[:, rows].T
+    assert np.allclose(lg, ref["lse"], rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("n,h_q,h_kv", [(1024, 32, 2), (777, 4, 1), (64, 16, 2), (1, 2, 1), (130, 8, 2)])
+def test_dense_attn_matches_oracle(n, h_q, h_kv):
+    sh, d = _problem(n, h_q, h_kv, k=64, seed=17)
+    op = oracle.params(sh)
+    p = infv2.params_of(sh)
+    rows = _sample_rows(n, 100)
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows)
+    lse = torch.empty((h_q, n), device="cuda")
+    o = infv2.infv2_dense_attn(p, to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]), lse=lse)
+    torch.cuda.synchronize()
+    og = synth.bf16_to_f32(to_host_bits(o))[rows]
+    parity.assert_outputs_close(og, ref["o"], "dense_attn")
+    assert np.allclose(lse.cpu().numpy()[:, rows].T, ref["lse"], rtol=0, atol=2e-3)
+
+
+def test_timeout_path_reports_and_recovers():
+    assert infv2.infv2_device_status() == 0
+    infv2.infv2_selftest_timeout(2000)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == infv2.ERR_TIMEOUT
+    assert infv2.infv2_device_status() == 0     # cleared
+    x = torch.ones(4, device="cuda") * 2        # the context is still usable
+    assert float(x.sum()) == 8.0

@@ -1,0 +1,27 @@
+// Launch functions shared between the library's translation units.
+#pragma once
+#include "common.cuh"
+
+namespace infv2 {
+
+int launch_compress_k(const uint16_t* k, int n, int h_kv, uint16_t* kc1, cudaStream_t st);
+
+int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
+                        int q_begin, int q_len, float* s_shared, int ld, float* score_lse,
+                        cudaStream_t st);
+
+int launch_select(const infv2_params* p, const float* s_shared, int ld, int n, int q_begin,
+                  int q_len, int* idx, long long idx_hstride, cudaStream_t st);
+
+// Row pitch (floats) of S^shared for an n-token sequence: at least the kernel
+// count and four kernels per block, rounded to 32 floats (128 bytes).
+inline int shared_ld(int n) {
+  const int nc = n >= 32 ? (n - 32) / 16 + 1 : 0;
+  const int nb = (n + 63) / 64;
+  int ld = nc > 4 * nb ? nc : 4 * nb;
+  return ((ld + 31) / 32) * 32;
+}
+
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace infv2

@@ -1,0 +1,319 @@
+// Stage 2: fused two-pass block scores (S^C1 softmax + GQA group sum).
+//
+// "InfLLM-V2" paper notes, key design 4, and the arXiv summary, section 3
+// ("Efficient Implementation"): S^C1 = softmax(Q K^C1^T) is never written to
+// memory; the head-group sum is taken on chip.  Because the group sum and the
+// online softmax do not commute, pass 1 computes each (token, head) row's
+// log-sum-exp and pass 2 recomputes the logits, normalises and sums over the
+// group; only S^shared (h_q/G values per token and kernel) reaches HBM.
+//
+// B200 design.  One CTA owns a tile of 128 (token, head) rows: TQ = 128/G
+// consecutive tokens times the G heads of kv head g (all heads of a group
+// share K^C1).  The Q tile (128 x 128 bf16) is loaded once by TMA and serves
+// both passes; K^C1 tiles of 128 kernels stream through a 4-stage TMA ring.
+//   pass 1: D[row, kernel]   = Q_tile . K^C1_tile^T   (tcgen05, M=128, N=128)
+//           one TMEM lane per row -> the row's running max / sum stay in one
+//           thread; lse2 (log2 domain) goes to shared memory.
+//   pass 2: D[kernel, row]   = K^C1_tile . Q_tile^T   (same operands swapped)
+//           one TMEM lane per kernel -> the G-head sum of exp2(z - lse2) for a
+//           token is a sum over G adjacent columns inside one thread, and the
+//           128 lanes store 128 consecutive floats of S^shared per token.
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps
+// 2-5 softmax / epilogue.  Accumulators are double-buffered in TMEM (2 x 128
+// columns) so the next tile's MMA overlaps the current tile's epilogue.
+#include "common.cuh"
+#include "internal.cuh"
+
+namespace infv2 {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct ScoreArgs {
+  int q_begin, q_len, n_tiles;
+  float scale_log2;     // scale * log2(e)
+  int ld;
+  float* s_shared;      // [h_kv, q_len, ld]
+  float* score_lse;     // [h_q, q_len] or null
+  WaitCtx wait;
+};
+
+struct ScoreSmem {
+  uint32_t q, k;        // shared addresses of the Q tile and the K^C1 ring
+  uint32_t q_full, kv_full, kv_empty, acc_full, acc_empty, lse_ready;  // barriers (8 B each)
+};
+
+template <int G>
+__global__ void __launch_bounds__(192, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 ScoreArgs a) {
+  constexpr int TQ = 128 / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  float* s_lse2 = reinterpret_cast<float*>(base + kTileBytes * (1 + kStages));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_lse2 + 128);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4);
+  ScoreSmem S;
+  S.q = smem_u32(base);
+  S.k = S.q + kTileBytes;
+  S.q_full = smem_u32(bars);
+  S.kv_full = S.q_full + 8;
+  S.kv_empty = S.kv_full + 8 * kStages;
+  S.acc_full = S.kv_empty + 8 * kStages;
+  S.acc_empty = S.acc_full + 16;
+  S.lse_ready = S.acc_empty + 16;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.y;
+  const int tile = a.n_tiles - 1 - (int)blockIdx.x;  // longest rows first
+  const int i0 = a.q_begin + tile * TQ;
+  const int i_last = min(i0 + TQ, a.q_begin + a.q_len) - 1;
+  const int nv_max = visible_kernels(i_last, 32, 16);
+  const int n_kt = (nv_max + 127) >> 7;
+
+  if (n_kt == 0) {  // no row of this tile sees a complete kernel
+    if (a.score_lse && threadIdx.x < 128) {
+      const int i = i0 + (int)threadIdx.x / G;
+      if (i <= i_last)
+        a.score_lse[(size_t)(g * G + threadIdx.x % G) * a.q_len + (i - a.q_begin)] = -INFINITY;
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(S.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(S.kv_full + 8 * s, 1);
+      mbar_init(S.kv_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(S.acc_full + 8 * b, 1);
+      mbar_init(S.acc_empty + 8 * b, 4);
+    }
+    mbar_init(S.lse_ready, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const int total_it = 2 * n_kt;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      mbar_expect_tx(S.q_full, kTileBytes);
+      tma_load_3d(S.q, &tm_q, S.q_full, 0, g * G, i0);
+      tma_load_3d(S.q + kTileBytes / 2, &tm_q, S.q_full, 64, g * G, i0);
+      int issued = 0;
+      for (int it = 0; it < total_it; ++it) {
+        const int s = it % kStages;
+        const int jt = it < n_kt ? it : it - n_kt;
+        if (!mbar_wait(S.kv_empty + 8 * s, ((it / kStages) & 1) ^ 1, a.wait)) break;
+        const uint32_t dst = S.k + s * kTileBytes;
+        mbar_expect_tx(S.kv_full + 8 * s, kTileBytes);
+        tma_load_3d(dst, &tm_k, S.kv_full + 8 * s, 0, g, jt * 128);
+        tma_load_3d(dst + kTileBytes / 2, &tm_k, S.kv_full + 8 * s, 64, g, jt * 128);
+        issued = it + 1;
+      }
+      // never leave a copy in flight: wait (bounded) for the last loads to land
+      (void)mbar_wait(S.q_full, 0, a.wait);
+      for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
+        (void)mbar_wait(S.kv_full + 8 * (it % kStages), (it / kStages) & 1, a.wait);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      bool ok = mbar_wait(S.q_full, 0, a.wait);
+      int issued = 0;
+      for (int it = 0; ok && it < total_it; ++it) {
+        const int s = it % kStages;
+        const int b = it & 1;
+        if (!mbar_wait(S.kv_full + 8 * s, (it / kStages) & 1, a.wait)) break;
+        if (!mbar_wait(S.acc_empty + 8 * b, ((it >> 1) & 1) ^ 1, a.wait)) break;
+        tc_fence_after();
+        const uint32_t ks = S.k + s * kTileBytes;
+        const uint32_t a_base = it < n_kt ? S.q : ks;   // pass 1: rows = Q; pass 2: rows = K^C1
+        const uint32_t b_base = it < n_kt ? ks : S.q;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+          umma_bf16_ss(tmem + b * 128, desc_kmajor_sw128(a_base + off),
+                       desc_kmajor_sw128(b_base + off), idesc, kk > 0);
+        }
+        umma_commit(S.kv_empty + 8 * s);
+        umma_commit(S.acc_full + 8 * b);
+        issued = it + 1;
+      }
+      // never free TMEM under a running MMA: wait (bounded) for the last commits
+      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
+        (void)mbar_wait(S.acc_full + 8 * (it & 1), (it >> 1) & 1, a.wait);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue warps
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int tq_r = r / G;
+    const int i_r = i0 + tq_r;
+    const int nv_r = i_r <= i_last ? visible_kernels(i_r, 32, 16) : 0;
+    const float c = a.scale_log2;
+    float vmax = -INFINITY, l = 0.f;
+    float* out_g = a.s_shared + (size_t)g * a.q_len * a.ld;
+    for (int it = 0; it < total_it; ++it) {
+      const int b = it & 1;
+      if (!mbar_wait(S.acc_full + 8 * b, (it >> 1) & 1, a.wait)) break;
+      tc_fence_after();
+      const uint32_t tb = lane_base + b * 128;
+      if (it < n_kt) {
+        // pass 1: row r, kernels it*128 .. +127
+        const int j0 = it * 128;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          float v[32];
+          tmem_ld32(tb + ch * 32, v);
+          tmem_ld_wait();
+          const int jb = j0 + ch * 32;
+          if (jb + 32 > nv_r) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (jb + e >= nv_r) v[e] = -INFINITY;
+          }
+          float cm = v[0];
+#pragma unroll
+          for (int e = 1; e < 32; ++e) cm = fmaxf(cm, v[e]);
+          if (cm > vmax) {
+            l *= fast_exp2((vmax - cm) * c);
+            vmax = cm;
+          }
+          if (vmax != -INFINITY) {
+            const float mneg = -vmax * c;
+            float part = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) part += fast_exp2(fmaf(v[e], c, mneg));
+            l += part;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);
+        if (it == n_kt - 1) {
+          const float lse2 = l > 0.f ? vmax * c + __log2f(l) : -INFINITY;
+          s_lse2[r] = lse2;
+          if (a.score_lse && i_r <= i_last)
+            a.score_lse[(size_t)(g * G + r % G) * a.q_len + (i_r - a.q_begin)] = lse2 * kLn2;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(S.lse_ready);
+          if (!mbar_wait(S.lse_ready, 0, a.wait)) break;  // all 128 rows' lse2 are in smem
+        }
+      } else {
+        // pass 2: kernel j = (it - n_kt)*128 + r, columns = (token, head)
+        const int j = (it - n_kt) * 128 + r;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          float v[32];
+          tmem_ld32(tb + ch * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 32 / G; ++t) {
+            const int tq = ch * (32 / G) + t;
+            const int i = i0 + tq;
+            float ssum = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+              ssum += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
+            if (i <= i_last && j < visible_kernels(i, 32, 16))
+              out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int G>
+int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h_kv, int q_begin,
+                   int q_len, float scale, float* s_shared, int ld, float* score_lse,
+                   cudaStream_t st) {
+  constexpr int TQ = 128 / G;
+  const int nc = n >= 32 ? (n - 32) / 16 + 1 : 0;
+  CUtensorMap tm_q, tm_k;
+  if (!make_tmap_3d(&tm_q, q, 128, h_q, n, 256, (uint64_t)h_q * 256, 64, G, TQ))
+    return INFV2_ERR_CUDA;
+  // K^C1 map; an empty K^C1 (nc == 0) still needs a valid map, one row is enough
+  if (!make_tmap_3d(&tm_k, kc1, 128, h_kv, nc > 0 ? nc : 1, 256, (uint64_t)h_kv * 256, 64, 1, 128))
+    return INFV2_ERR_CUDA;
+  const int smem = kTileBytes * (1 + kStages) + 128 * 4 + 8 * (2 + 2 * kStages + 4) + 16 + 1024;
+  if (!set_smem(score_kernel<G>, smem)) return INFV2_ERR_CUDA;
+  ScoreArgs a;
+  a.q_begin = q_begin;
+  a.q_len = q_len;
+  a.n_tiles = (q_len + TQ - 1) / TQ;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.ld = ld;
+  a.s_shared = s_shared;
+  a.score_lse = score_lse;
+  a.wait = wait_ctx();
+  dim3 grid(a.n_tiles, h_kv);
+  score_kernel<G><<<grid, 192, smem, st>>>(tm_q, tm_k, a);
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
+                        int q_begin, int q_len, float* s_shared, int ld, float* score_lse,
+                        cudaStream_t st) {
+  if (q_len <= 0) return INFV2_OK;
+  const int G = p->h_q / p->h_kv;
+  switch (G) {
+    case 1: return launch_score_g<1>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
+    case 2: return launch_score_g<2>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
+    case 4: return launch_score_g<4>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
+    case 8: return launch_score_g<8>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
+    case 16: return launch_score_g<16>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
+    default: return INFV2_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace infv2
+
+using namespace infv2;
+
+extern "C" int infv2_block_scores(const infv2_params* p, const void* q, const void* kc1, int n,
+                                  int q_begin, int q_len, float* s_shared, int ld,
+                                  float* score_lse, infv2_stream_t stream) {
+  int st = infv2_check_params(p);
+  if (st != INFV2_OK) return st;
+  if (n < 0 || q_begin < 0 || q_len < 0 || q_begin + q_len > n) return INFV2_ERR_INVALID_ARG;
+  if (q_len == 0) return INFV2_OK;
+  if (!q || !s_shared) return INFV2_ERR_INVALID_ARG;
+  const int nc = infv2_num_kernels(p, n);
+  if (nc > 0 && !kc1) return INFV2_ERR_INVALID_ARG;
+  if (ld < nc || ld % 4 != 0) return INFV2_ERR_INVALID_ARG;
+  if (nc == 0 && score_lse == nullptr) return INFV2_OK;
+  const void* kc1_map = kc1 ? kc1 : q;  // any valid address when no kernel exists
+  return launch_block_scores(p, static_cast<const uint16_t*>(q),
+                             static_cast<const uint16_t*>(kc1_map), n, q_begin, q_len, s_shared,
+                             ld, score_lse, reinterpret_cast<cudaStream_t>(stream));
+}

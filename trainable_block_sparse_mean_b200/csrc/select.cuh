@@ -1,0 +1,137 @@
+// Stages 3-4 for one (query, kv head) row, executed by one warp: max pooling
+// of S^shared into block scores and the top-k block selection.
+//
+// "InfLLM-V2" paper notes, key designs 2-3, and the MiniCPM4 "InfLLM v2" blog
+// (semantic kernels, top-k sharing):
+//   S^cmp[b] = max over the visible kernels j that intersect block b (with
+//              B=64, l_C1=32, s_C1=16 these are j = 4b-1 .. 4b+3);
+//   I(i)     = every block 0..i/B when there are at most k of them; otherwise
+//              the init and local blocks (treated as +inf) plus the highest
+//              S^cmp blocks up to k in total, equal scores to the lower block.
+// The selection is an exact radix select on order-preserving 32-bit keys: four
+// 8-bit digit passes with a per-warp shared-memory histogram find the k-th
+// largest key T; blocks with key > T are taken, and the blocks with key == T
+// are taken in ascending block order until k are chosen.
+#pragma once
+#include "common.cuh"
+
+namespace infv2 {
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr uint32_t kForcedKey = 0xFFFFFFFFu;  // above every finite score and +inf
+
+// Select for one row.  `row` holds S^shared[j] for j < nv (entries at
+// j >= nv may be garbage and are never used; reads stay below 4*(bi+1)).
+// `keys` is per-warp shared scratch of >= bi+1 words, `hist` 256 words.
+// Writes k indices (ascending, -1 padded) to `out`.
+__device__ __forceinline__ void select_row_warp(const float* __restrict__ row, int nv, int i,
+                                                int n_init, int n_local, int k, uint32_t* keys,
+                                                uint32_t* hist, int* __restrict__ out) {
+  const int lane = (int)lane_id();
+  const int bi = i >> 6;  // own block (B = 64)
+  const int n_cand = bi + 1;
+  if (n_cand <= k) {  // dense: every visible block
+    for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
+    return;
+  }
+  // ---- max pooling into order keys (forced blocks get the top key)
+  float carry = -INFINITY;  // S^shared[4*base - 1] for the next chunk's lane 0
+  for (int base = 0; base < n_cand; base += 32) {
+    const int b = base + lane;
+    float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    const int j0 = 4 * b;
+    if (b < n_cand) {
+      if (j0 + 3 < nv) {
+        v = *reinterpret_cast<const float4*>(row + j0);
+      } else {
+        if (j0 + 0 < nv) v.x = row[j0 + 0];
+        if (j0 + 1 < nv) v.y = row[j0 + 1];
+        if (j0 + 2 < nv) v.z = row[j0 + 2];
+      }
+    }
+    // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
+    float prev = __shfl_up_sync(0xFFFFFFFFu, v.w, 1);
+    if (lane == 0) prev = carry;
+    carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
+    if (b < n_cand) {
+      const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
+      const bool forced = b < n_init || b > bi - n_local;
+      keys[b] = forced ? kForcedKey : float_key(m);
+    }
+  }
+  __syncwarp();
+  // ---- radix select of the k-th largest key
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int x = lane; x < 256; x += 32) hist[x] = 0;
+    __syncwarp();
+    for (int b = lane; b < n_cand; b += 32) {
+      const uint32_t key = keys[b];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane L owns digits 255-8L .. 248-8L (lane 0 the largest)
+    uint32_t cnt[8];
+    uint32_t local = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      cnt[e] = hist[255 - 8 * lane - e];
+      local += cnt[e];
+    }
+    uint32_t incl = local;  // inclusive scan over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const uint32_t before = incl - local;
+    const bool mine = before < (uint32_t)remaining && (uint32_t)remaining <= incl;
+    uint32_t digit = 0, above = 0;
+    if (mine) {
+      uint32_t run = before;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (run + cnt[e] >= (uint32_t)remaining) {
+          digit = 255u - 8u * lane - e;
+          above = run;
+          break;
+        }
+        run += cnt[e];
+      }
+    }
+    const uint32_t who = __ballot_sync(0xFFFFFFFFu, mine);
+    const int src = __ffs(who) - 1;
+    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
+    above = __shfl_sync(0xFFFFFFFFu, above, src);
+    prefix |= digit << shift;
+    pmask |= 255u << shift;
+    remaining -= (int)above;
+    __syncwarp();
+  }
+  // ---- emit ascending: key > T, then key == T in block order while needed
+  const uint32_t T = prefix;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int eq_seen = 0, written = 0;
+  for (int base = 0; base < n_cand; base += 32) {
+    const int b = base + lane;
+    const uint32_t key = b < n_cand ? keys[b] : 0u;
+    const bool eq = b < n_cand && key == T;
+    const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
+    const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
+    eq_seen += __popc(eqb);
+    const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) out[written + __popc(selb & lt_mask)] = b;
+    written += __popc(selb);
+  }
+  for (int x = written + lane; x < k; x += 32) out[x] = -1;
+  __syncwarp();
+}
+
+}  // namespace infv2

@@ -1,0 +1,230 @@
+"""Thin Python binding of libinfv2.so (argument marshalling only).
+
+Every function has the name of the C entry point it calls and takes torch
+CUDA tensors; all computation happens in the library's kernels.  A missing
+library or a non-zero status raises.  Nothing here falls back to the CPU.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libinfv2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+
+SYMBOLS = [
+    "infv2_default_params", "infv2_check_params", "infv2_status_string", "infv2_num_kernels",
+    "infv2_device_status", "infv2_compress_k", "infv2_block_scores", "infv2_select_topk",
+    "infv2_sparse_attn", "infv2_dense_attn", "infv2_prefill_workspace_size", "infv2_prefill",
+    "infv2_decode_workspace_size", "infv2_decode", "infv2_selftest_timeout",
+]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("l_c1", ctypes.c_int), ("s_c1", ctypes.c_int),
+                ("pool_l", ctypes.c_int), ("pool_s", ctypes.c_int), ("n_init", ctypes.c_int),
+                ("n_local", ctypes.c_int), ("k", ctypes.c_int), ("h_q", ctypes.c_int),
+                ("h_kv", ctypes.c_int), ("d", ctypes.c_int), ("scale", ctypes.c_float),
+                ("window", ctypes.c_int)]
+
+
+class Infv2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__("%s failed: %s (status %d)" % (where, status_string(status), status))
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libinfv2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libinfv2.so not built: run python -m trainable_block_sparse_mean_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(Params)
+        vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.infv2_default_params.argtypes = [P, i, i]
+        L.infv2_default_params.restype = None
+        L.infv2_check_params.argtypes = [P]
+        L.infv2_status_string.argtypes = [i]
+        L.infv2_status_string.restype = ctypes.c_char_p
+        L.infv2_num_kernels.argtypes = [P, i]
+        L.infv2_device_status.argtypes = [vp]
+        L.infv2_compress_k.argtypes = [P, vp, i, vp, vp]
+        L.infv2_block_scores.argtypes = [P, vp, vp, i, i, i, vp, i, vp, vp]
+        L.infv2_select_topk.argtypes = [P, vp, i, i, i, i, vp, vp]
+        L.infv2_sparse_attn.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
+        L.infv2_dense_attn.argtypes = [P, vp, vp, vp, i, vp, vp, vp]
+        L.infv2_prefill_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
+        L.infv2_prefill.argtypes = [P, vp, vp, vp, vp, i, vp, sz, vp, vp, vp, vp]
+        L.infv2_decode_workspace_size.argtypes = [P, i, i, ctypes.POINTER(sz)]
+        L.infv2_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i, i, vp, sz, vp, vp, vp, vp]
+        L.infv2_selftest_timeout.argtypes = [i, vp]
+        _lib = L
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return lib().infv2_status_string(st).decode()
+
+
+def _check(st: int, where: str):
+    if st != OK:
+        raise Infv2Error(st, where)
+
+
+def params(h_q: int, h_kv: int, k: int = 64, n_init: int = 1, n_local: int = 2,
+           scale: float | None = None, window: int = 0) -> Params:
+    p = Params()
+    lib().infv2_default_params(ctypes.byref(p), h_q, h_kv)
+    p.k, p.n_init, p.n_local, p.window = k, n_init, n_local, window
+    if scale is not None:
+        p.scale = scale
+    return p
+
+
+def params_of(shape) -> Params:
+    """Library parameters from a synth.Shape."""
+    p = params(shape.h_q, shape.h_kv, k=shape.k, n_init=shape.n_init, n_local=shape.n_local)
+    p.B, p.l_c1, p.s_c1, p.pool_l, p.pool_s, p.d = (shape.B, shape.l_c1, shape.s_c1,
+                                                   shape.pool_l, shape.pool_s, shape.d)
+    p.scale = 1.0 / math.sqrt(shape.d)
+    return p
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def num_kernels(p: Params, n: int) -> int:
+    return lib().infv2_num_kernels(ctypes.byref(p), n)
+
+
+def shared_ld(n: int) -> int:
+    """Row pitch of S^shared: >= kernel count and 4 kernels per block, x32."""
+    nc = (n - 32) // 16 + 1 if n >= 32 else 0
+    nb = (n + 63) // 64
+    return ((max(nc, 4 * nb) + 31) // 32) * 32
+
+
+def infv2_check_params(p: Params) -> int:
+    return lib().infv2_check_params(ctypes.byref(p))
+
+
+def infv2_device_status(stream=None) -> int:
+    return lib().infv2_device_status(_stream(stream))
+
+
+def infv2_compress_k(p: Params, k: torch.Tensor, kc1: torch.Tensor | None = None, stream=None):
+    n = k.shape[0]
+    if kc1 is None:
+        kc1 = torch.empty((max(num_kernels(p, n), 0), p.h_kv, p.d), dtype=torch.bfloat16,
+                          device=k.device)
+    _check(lib().infv2_compress_k(ctypes.byref(p), _ptr(k), n, _ptr(kc1) if kc1.numel() else None,
+                                  _stream(stream)), "infv2_compress_k")
+    return kc1
+
+
+def infv2_block_scores(p: Params, q, kc1, n: int, q_begin: int, q_len: int, s_shared=None,
+                       ld: int | None = None, score_lse=None, stream=None):
+    ld = shared_ld(n) if ld is None else ld
+    if s_shared is None:
+        s_shared = torch.zeros((p.h_kv, q_len, ld), dtype=torch.float32, device=q.device)
+    _check(lib().infv2_block_scores(ctypes.byref(p), _ptr(q), _ptr(kc1) if kc1.numel() else None,
+                                    n, q_begin, q_len, _ptr(s_shared), ld, _ptr(score_lse),
+                                    _stream(stream)), "infv2_block_scores")
+    return s_shared
+
+
+def infv2_select_topk(p: Params, s_shared, ld: int, n: int, q_begin: int, q_len: int, idx=None,
+                      stream=None):
+    if idx is None:
+        idx = torch.full((p.h_kv, n, p.k), -2, dtype=torch.int32, device=s_shared.device)
+    _check(lib().infv2_select_topk(ctypes.byref(p), _ptr(s_shared), ld, n, q_begin, q_len,
+                                   _ptr(idx), _stream(stream)), "infv2_select_topk")
+    return idx
+
+
+def infv2_sparse_attn(p: Params, q, k, v, idx, o=None, lse=None, stream=None):
+    n = q.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_sparse_attn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), n,
+                                   _ptr(o), _ptr(lse), _stream(stream)), "infv2_sparse_attn")
+    return o
+
+
+def infv2_dense_attn(p: Params, q, k, v, o=None, lse=None, stream=None):
+    n = q.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_dense_attn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), n, _ptr(o),
+                                  _ptr(lse), _stream(stream)), "infv2_dense_attn")
+    return o
+
+
+def infv2_prefill_workspace_size(p: Params, cu_seqlens) -> int:
+    cu = (ctypes.c_int * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    out = ctypes.c_size_t(0)
+    _check(lib().infv2_prefill_workspace_size(ctypes.byref(p), ctypes.cast(cu, ctypes.c_void_p),
+                                              len(cu_seqlens) - 1, ctypes.byref(out)),
+           "infv2_prefill_workspace_size")
+    return out.value
+
+
+def infv2_prefill(p: Params, q, k, v, cu_seqlens, workspace=None, idx_out=None, o=None, lse=None,
+                  stream=None):
+    """Whole layer over a packed varlen batch; cu_seqlens is a host sequence."""
+    cu = (ctypes.c_int * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    need = infv2_prefill_workspace_size(p, cu_seqlens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                               ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1,
+                               _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(o),
+                               _ptr(lse), _stream(stream)), "infv2_prefill")
+    return o
+
+
+def infv2_decode_workspace_size(p: Params, batch: int, cap: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().infv2_decode_workspace_size(ctypes.byref(p), batch, cap, ctypes.byref(out)),
+           "infv2_decode_workspace_size")
+    return out.value
+
+
+def infv2_decode(p: Params, q, k_new, v_new, k_cache, v_cache, kc1_cache, seqlens, workspace,
+                 idx_out=None, o=None, lse=None, stream=None):
+    batch, cap = k_cache.shape[0], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_decode(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                              _ptr(v_cache), _ptr(kc1_cache), _ptr(seqlens), batch, cap,
+                              _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(o),
+                              _ptr(lse), _stream(stream)), "infv2_decode")
+    return o
+
+
+def infv2_selftest_timeout(limit_us: int, stream=None):
+    _check(lib().infv2_selftest_timeout(limit_us, _stream(stream)), "infv2_selftest_timeout")
