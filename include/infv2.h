@@ -23,7 +23,8 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, unless a
  *     parameter says "host".  The library allocates no memory; scratch space
- *     is the caller's `workspace`.
+ *     is the caller's `workspace` (infv2_select_blocks_noalloc instead uses a
+ *     fixed array that the library holds on each device).
  *   - bf16 tensors are raw 16-bit patterns (e.g. torch.bfloat16 storage);
  *     every tensor is dense, row-major, 16-byte aligned.
  *   - Token layout ("thd"): q [n, h_q, d], k and v [n, h_kv, d]; query head h
@@ -188,6 +189,27 @@ int infv2_decode(const infv2_params* p, const void* q, const void* k_new, const 
                  void* k_cache, void* v_cache, void* kc1_cache, int* seqlens, int batch, int cap,
                  void* workspace, size_t ws_bytes, int* idx_out, void* o, float* lse,
                  infv2_stream_t stream);
+
+/* Block selection (the work of infv2_block_scores followed by
+ * infv2_select_topk) for callers that cannot allocate device memory: code that
+ * runs inside a memory arena or pool it does not own, an engine whose
+ * allocator is frozen after start-up, or a plugin that only receives input and
+ * output pointers.  The paper has no counterpart; this is a packaging variant.
+ * The intermediate S^shared rows live in a 16 MiB array that the library
+ * keeps on every GPU that loads it until the process exits; nothing is
+ * allocated and no workspace is taken.  Inputs and output are as for the two
+ * calls it replaces:
+ *   q    bf16 [n, h_q, d];  kc1  bf16 [num_kernels(n), h_kv, d]
+ *   idx  int32 [h_kv, n, k] (output): rows q_begin .. q_begin+q_len-1 written.
+ * Rows are processed in chunks that fit the array.  Sizes whose S^shared rows
+ * for one 128-token tile do not fit (h_kv * ld * 4 * 128 > 16 MiB, with
+ * ld = max(num_kernels(n), 4*ceil(n/B)) rounded up to 32; e.g. n > 262144 at
+ * h_kv = 2) return INFV2_ERR_UNSUPPORTED.  The first call on a device looks up
+ * the array's device address (make it before any stream capture).  Every call
+ * shares the array: calls that can overlap on the GPU race and must be
+ * serialised by the caller. */
+int infv2_select_blocks_noalloc(const infv2_params* p, const void* q, const void* kc1, int n,
+                                int q_begin, int q_len, int* idx, infv2_stream_t stream);
 
 /* Self-test of the bounded-wait error path: launches one kernel that waits
  * on a barrier nobody arrives at, with the given limit in microseconds; the

@@ -21,7 +21,8 @@ SYMBOLS = [
     "infv2_default_params", "infv2_check_params", "infv2_status_string", "infv2_num_kernels",
     "infv2_device_status", "infv2_compress_k", "infv2_block_scores", "infv2_select_topk",
     "infv2_sparse_attn", "infv2_dense_attn", "infv2_prefill_workspace_size", "infv2_prefill",
-    "infv2_decode_workspace_size", "infv2_decode", "infv2_selftest_timeout",
+    "infv2_decode_workspace_size", "infv2_decode", "infv2_select_blocks_noalloc",
+    "infv2_selftest_timeout",
 ]
 
 
@@ -67,6 +68,7 @@ def lib():
         L.infv2_prefill.argtypes = [P, vp, vp, vp, vp, i, vp, sz, vp, vp, vp, vp]
         L.infv2_decode_workspace_size.argtypes = [P, i, i, ctypes.POINTER(sz)]
         L.infv2_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i, i, vp, sz, vp, vp, vp, vp]
+        L.infv2_select_blocks_noalloc.argtypes = [P, vp, vp, i, i, i, vp, vp]
         L.infv2_selftest_timeout.argtypes = [i, vp]
         _lib = L
     return _lib
@@ -224,6 +226,16 @@ def infv2_decode(p: Params, q, k_new, v_new, k_cache, v_cache, kc1_cache, seqlen
                               _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(o),
                               _ptr(lse), _stream(stream)), "infv2_decode")
     return o
+
+
+def infv2_select_blocks_noalloc(p: Params, q, kc1, n: int, q_begin: int, q_len: int, idx,
+                                stream=None):
+    """Block selection with the library's fixed device scratch (no allocation)."""
+    _check(lib().infv2_select_blocks_noalloc(ctypes.byref(p), _ptr(q),
+                                             _ptr(kc1) if kc1.numel() else None, n, q_begin,
+                                             q_len, _ptr(idx), _stream(stream)),
+           "infv2_select_blocks_noalloc")
+    return idx
 
 
 def infv2_selftest_timeout(limit_us: int, stream=None):
