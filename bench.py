@@ -177,7 +177,7 @@ def run_ours(args, rank, world, local_rank, dist):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    shape = synth.CONFIGS["c3"]["shape"]
+    shape = synth.CONFIGS[args.workload]["shape"]
     n = shape.n
     p = infv2.params_of(shape)
     data = synth.make_prefill(shape, seed=rank)
@@ -227,6 +227,9 @@ def run_ours(args, rank, world, local_rank, dist):
     n_chunks = (n + chunk_rows - 1) // chunk_rows
     launches_per_step = 1 + 2 * n_chunks + 1
 
+    if args.only == "prefill":   # profiling runs: the timed prefill steps only
+        return {"metric": METRIC, "ms_per_step": round(ms, 4), "workload": args.workload,
+                "launches_per_step": launches_per_step}
     # ---- per-stage breakdown on the same stream (CUDA events between launches)
     stage = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows)
     # ---- end to end through host buffers
@@ -515,6 +518,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["c3", "c2"], default="c3",
+                    help="prefill workload: c3 (131072 tokens, the reported one) or c2 (32768)")
+    ap.add_argument("--only", choices=["all", "prefill"], default="all",
+                    help="prefill: time the prefill steps only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -543,7 +550,7 @@ def main():
         dist.barrier()
     try:
         out = run_ours(args, rank, world, local_rank, dist)
-        if rank == 0 and not args.no_cpu_baseline:
+        if rank == 0 and not args.no_cpu_baseline and args.only == "all":
             cpu, _, _ = oracle_sample()
             out["cpu_baseline"] = cpu
         if rank == 0:
