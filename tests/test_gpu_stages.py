@@ -140,7 +140,8 @@ def test_select_exact_on_oracle_scores(n, h_q, h_kv, k):
 
 # ---------------------------------------------------------------- stage 5
 
-@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (3001, 32, 2, 16), (1500, 16, 2, 4)])
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (2048, 16, 1, 8), (3001, 32, 2, 16),
+                                         (1500, 16, 2, 4)])
 def test_sparse_attn_on_oracle_indices(n, h_q, h_kv, k):
     sh, d = _problem(n, h_q, h_kv, k=k, seed=11)
     op = oracle.params(sh)
@@ -150,15 +151,21 @@ def test_sparse_attn_on_oracle_indices(n, h_q, h_kv, k):
     idx = np.full((h_kv, n, k), -1, np.int32)
     idx[:, :, 0] = (np.arange(n) // 64)[None, :]   # rows not sampled: own block only
     idx[:, rows, :] = ref["idx"].transpose(1, 0, 2)
-    lse = torch.empty((h_q, n), device="cuda")
-    o = infv2.infv2_sparse_attn(p, to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]),
-                                torch.from_numpy(idx).cuda(), lse=lse)
-    torch.cuda.synchronize()
-    assert infv2.infv2_device_status() == 0
-    og = synth.bf16_to_f32(to_host_bits(o))[rows]
-    parity.assert_outputs_close(og, ref["o"], "sparse_attn")
-    lg = lse.cpu().numpy()[:, rows].T
-    assert np.allclose(lg, ref["lse"], rtol=0, atol=2e-3)
+    q, kk, vv, ii = to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]), torch.from_numpy(idx).cuda()
+    first = None
+    for rep in range(3):   # repeated launches: a pipeline race shows up as run-to-run change
+        lse = torch.empty((h_q, n), device="cuda")
+        o = infv2.infv2_sparse_attn(p, q, kk, vv, ii, lse=lse)
+        torch.cuda.synchronize()
+        assert infv2.infv2_device_status() == 0
+        og = synth.bf16_to_f32(to_host_bits(o))[rows]
+        parity.assert_outputs_close(og, ref["o"], "sparse_attn")
+        lg = lse.cpu().numpy()[:, rows].T
+        assert np.allclose(lg, ref["lse"], rtol=0, atol=2e-3)
+        if first is None:
+            first = og
+        else:
+            assert np.array_equal(og, first), "sparse_attn is not deterministic"
 
 
 @pytest.mark.parametrize("n,h_q,h_kv", [(1024, 32, 2), (777, 4, 1), (64, 16, 2), (1, 2, 1), (130, 8, 2)])

@@ -25,8 +25,12 @@
 namespace infv2 {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 2;                // 2 stages -> two CTAs fit on one SM
 constexpr int kHalf = 64 * 64 * 2;        // 64 keys x 64 dims of bf16 = 8 KB
+// A row's reference max is only raised when a block's max exceeds it by more
+// than this (log2 units): probabilities stay below 2^8, and O, l are rescaled
+// rarely.  The final normalisation makes the result independent of it.
+constexpr float kRescaleSlack = 8.0f;
 constexpr int kStageBytes = 4 * kHalf;    // K (2 halves) + V (2 halves)
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -92,7 +96,7 @@ __device__ __forceinline__ void item_range(const AttnArgs& a, const Item& it, in
 
 __device__ __forceinline__ int block_at(const int* row, int e) { return row ? __ldg(row + e) : e; }
 
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(160, 2)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -222,28 +226,49 @@ __global__ void __launch_bounds__(160, 1)
           mma16816(sc[1], qa[ks], b2, b3);
         }
       }
-      // ---- causal mask and online softmax (rows gid and gid+8)
+      // ---- causal mask (only a block reaching past the query) and online
+      // softmax with a lazily raised reference max (rows gid and gid+8)
       const int t0 = 64 * b + kb;
       float z[2][4];
+      if (64 * b + 63 <= pos) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int t = t0 + nt * 8 + 2 * tig + (e2 & 1);
-          z[nt][e2] = t <= pos ? sc[nt][e2] * c : -INFINITY;
-        }
+          for (int e2 = 0; e2 < 4; ++e2) z[nt][e2] = sc[nt][e2] * c;
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int t = t0 + nt * 8 + 2 * tig + (e2 & 1);
+            z[nt][e2] = t <= pos ? sc[nt][e2] * c : -INFINITY;
+          }
+      }
       float mx0 = fmaxf(fmaxf(z[0][0], z[0][1]), fmaxf(z[1][0], z[1][1]));
       float mx1 = fmaxf(fmaxf(z[0][2], z[0][3]), fmaxf(z[1][2], z[1][3]));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
-      const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = fast_exp2(m0 - ref0), al1 = fast_exp2(m1 - ref1);
-      m0 = mn0;
-      m1 = mn1;
+      const bool raise = mx0 > m0 + kRescaleSlack || mx1 > m1 + kRescaleSlack;
+      if (__any_sync(0xFFFFFFFFu, raise)) {
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = mn0 == -INFINITY ? 1.f : fast_exp2(m0 - mn0);
+        const float al1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        l0 *= al0;
+        l1 *= al1;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          o[nt][0] *= al0;
+          o[nt][1] *= al0;
+          o[nt][2] *= al1;
+          o[nt][3] *= al1;
+        }
+      }
+      const float ref0 = m0 == -INFINITY ? 0.f : m0;
+      const float ref1 = m1 == -INFINITY ? 0.f : m1;
       float p[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
@@ -252,15 +277,8 @@ __global__ void __launch_bounds__(160, 1)
         p[nt][2] = fast_exp2(z[nt][2] - ref1);
         p[nt][3] = fast_exp2(z[nt][3] - ref1);
       }
-      l0 = l0 * al0 + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-      l1 = l1 * al1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        o[nt][0] *= al0;
-        o[nt][1] *= al0;
-        o[nt][2] *= al1;
-        o[nt][3] *= al1;
-      }
+      l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+      l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
       uint32_t pa[4];
       pa[0] = pack_bf16(p[0][0], p[0][1]);
       pa[1] = pack_bf16(p[0][2], p[0][3]);
@@ -280,6 +298,9 @@ __global__ void __launch_bounds__(160, 1)
           mma16816(o[nt + 1], pa, b2, b3);
         }
       }
+      // The stage was read through the generic proxy (ldmatrix) and will be
+      // rewritten by TMA (async proxy): order the two before releasing it.
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * s);
       ++cc;
@@ -377,7 +398,12 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
   if (n_items == 0) return INFV2_OK;
   const int smem = kStages * kStageBytes + (4 * 16 * 128 + 128) * 4 + 8 * (2 * kStages + 1) + 1024;
   if (!set_smem(sparse_attn_kernel, smem)) return INFV2_ERR_CUDA;
-  const long long grid = n_items < sm_count() ? n_items : sm_count();
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_attn_kernel, 160, smem) !=
+          cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const long long slots = (long long)per_sm * sm_count();
+  const long long grid = n_items < slots ? n_items : slots;
   sparse_attn_kernel<<<(unsigned)grid, 160, smem, st>>>(tm_k, tm_v, a);
   return launch_status(cudaGetLastError());
 }

@@ -19,8 +19,10 @@
 //           token is a sum over G adjacent columns inside one thread, and the
 //           128 lanes store 128 consecutive floats of S^shared per token.
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps
-// 2-5 softmax / epilogue.  Accumulators are double-buffered in TMEM (2 x 128
-// columns) so the next tile's MMA overlaps the current tile's epilogue.
+// 2-9 softmax / epilogue: two warpgroups, each owning 64 of a tile's 128
+// columns (pass-1 row statistics are merged through shared memory).
+// Accumulators are double-buffered in TMEM (2 x 128 columns) so the next
+// tile's MMA overlaps the current tile's epilogue.
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -29,6 +31,8 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
+constexpr int kEpiWarps = 8;               // two epilogue warpgroups
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct ScoreArgs {
@@ -46,7 +50,7 @@ struct ScoreSmem {
 };
 
 template <int G>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  ScoreArgs a) {
   constexpr int TQ = 128 / G;
@@ -54,7 +58,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   float* s_lse2 = reinterpret_cast<float*>(base + kTileBytes * (1 + kStages));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_lse2 + 128);
+  float* s_part = s_lse2 + 128;  // [2 halves][128 rows][max, sum]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + 2 * 128 * 2);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4);
   ScoreSmem S;
   S.q = smem_u32(base);
@@ -92,9 +97,9 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(S.acc_full + 8 * b, 1);
-      mbar_init(S.acc_empty + 8 * b, 4);
+      mbar_init(S.acc_empty + 8 * b, kEpiWarps);
     }
-    mbar_init(S.lse_ready, 4);
+    mbar_init(S.lse_ready, kEpiWarps);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -162,9 +167,10 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue warps
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
+    const int half = (warp - 2) >> 2;    // columns 64*half .. +63 of every tile
     const int r = quarter * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 64;
     const int tq_r = r / G;
     const int i_r = i0 + tq_r;
     const int nv_r = i_r <= i_last ? visible_kernels(i_r, 32, 16) : 0;
@@ -175,71 +181,79 @@ __global__ void __launch_bounds__(192, 1)
       const int b = it & 1;
       if (!mbar_wait(S.acc_full + 8 * b, (it >> 1) & 1, a.wait)) break;
       tc_fence_after();
-      const uint32_t tb = lane_base + b * 128;
+      float v[64];
+      {
+        float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+        float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+        tmem_ld32(lane_base + b * 128, v0);
+        tmem_ld32(lane_base + b * 128 + 32, v1);
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);  // TMEM buffer free again
       if (it < n_kt) {
-        // pass 1: row r, kernels it*128 .. +127
-        const int j0 = it * 128;
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          float v[32];
-          tmem_ld32(tb + ch * 32, v);
-          tmem_ld_wait();
-          const int jb = j0 + ch * 32;
-          if (jb + 32 > nv_r) {
+        // pass 1: row r, kernels it*128 + 64*half .. +63
+        const int jb = it * 128 + half * 64;
+        if (jb + 64 > nv_r) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (jb + e >= nv_r) v[e] = -INFINITY;
-          }
-          float cm = v[0];
-#pragma unroll
-          for (int e = 1; e < 32; ++e) cm = fmaxf(cm, v[e]);
-          if (cm > vmax) {
-            l *= fast_exp2((vmax - cm) * c);
-            vmax = cm;
-          }
-          if (vmax != -INFINITY) {
-            const float mneg = -vmax * c;
-            float part = 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) part += fast_exp2(fmaf(v[e], c, mneg));
-            l += part;
-          }
+          for (int e = 0; e < 64; ++e)
+            if (jb + e >= nv_r) v[e] = -INFINITY;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);
+        float cm = v[0];
+#pragma unroll
+        for (int e = 1; e < 64; ++e) cm = fmaxf(cm, v[e]);
+        if (cm > vmax) {
+          l *= fast_exp2((vmax - cm) * c);
+          vmax = cm;
+        }
+        if (vmax != -INFINITY) {
+          const float mneg = -vmax * c;
+          float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            p0 += fast_exp2(fmaf(v[e], c, mneg));
+            p1 += fast_exp2(fmaf(v[e + 1], c, mneg));
+          }
+          l += p0 + p1;
+        }
         if (it == n_kt - 1) {
-          const float lse2 = l > 0.f ? vmax * c + __log2f(l) : -INFINITY;
-          s_lse2[r] = lse2;
-          if (a.score_lse && i_r <= i_last)
-            a.score_lse[(size_t)(g * G + r % G) * a.q_len + (i_r - a.q_begin)] = lse2 * kLn2;
+          // merge the two column halves of row r
+          s_part[(half * 128 + r) * 2 + 0] = vmax;
+          s_part[(half * 128 + r) * 2 + 1] = l;
           __syncwarp();
           if (lane == 0) mbar_arrive(S.lse_ready);
-          if (!mbar_wait(S.lse_ready, 0, a.wait)) break;  // all 128 rows' lse2 are in smem
+          if (!mbar_wait(S.lse_ready, 0, a.wait)) break;
+          if (half == 0) {
+            const float m0 = s_part[r * 2], l0 = s_part[r * 2 + 1];
+            const float m1 = s_part[(128 + r) * 2], l1 = s_part[(128 + r) * 2 + 1];
+            const float M = fmaxf(m0, m1);
+            float L = 0.f;
+            if (m0 != -INFINITY) L += l0 * fast_exp2((m0 - M) * c);
+            if (m1 != -INFINITY) L += l1 * fast_exp2((m1 - M) * c);
+            const float lse2 = L > 0.f ? M * c + __log2f(L) : -INFINITY;
+            s_lse2[r] = lse2;
+            if (a.score_lse && i_r <= i_last)
+              a.score_lse[(size_t)(g * G + r % G) * a.q_len + (i_r - a.q_begin)] = lse2 * kLn2;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(S.lse_ready);
+          if (!mbar_wait(S.lse_ready, 1, a.wait)) break;  // all 128 lse2 in smem
         }
       } else {
-        // pass 2: kernel j = (it - n_kt)*128 + r, columns = (token, head)
+        // pass 2: kernel j = (it - n_kt)*128 + r; columns 64*half.. = tokens
         const int j = (it - n_kt) * 128 + r;
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          float v[32];
-          tmem_ld32(tb + ch * 32, v);
-          tmem_ld_wait();
 #pragma unroll
-          for (int t = 0; t < 32 / G; ++t) {
-            const int tq = ch * (32 / G) + t;
-            const int i = i0 + tq;
-            float ssum = 0.f;
+        for (int t = 0; t < 64 / G; ++t) {
+          const int tq = half * (64 / G) + t;
+          const int i = i0 + tq;
+          float ssum = 0.f;
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh)
-              ssum += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
-            if (i <= i_last && j < visible_kernels(i, 32, 16))
-              out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
-          }
+          for (int hh = 0; hh < G; ++hh)
+            ssum += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
+          if (i <= i_last && j < visible_kernels(i, 32, 16))
+            out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);
       }
     }
   }
@@ -263,7 +277,8 @@ int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h
   // K^C1 map; an empty K^C1 (nc == 0) still needs a valid map, one row is enough
   if (!make_tmap_3d(&tm_k, kc1, 128, h_kv, nc > 0 ? nc : 1, 256, (uint64_t)h_kv * 256, 64, 1, 128))
     return INFV2_ERR_CUDA;
-  const int smem = kTileBytes * (1 + kStages) + 128 * 4 + 8 * (2 + 2 * kStages + 4) + 16 + 1024;
+  const int smem = kTileBytes * (1 + kStages) + 128 * 4 + 2 * 128 * 2 * 4 + 8 * (2 + 2 * kStages + 4) +
+                   16 + 1024;
   if (!set_smem(score_kernel<G>, smem)) return INFV2_ERR_CUDA;
   ScoreArgs a;
   a.q_begin = q_begin;
@@ -275,7 +290,7 @@ int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h
   a.score_lse = score_lse;
   a.wait = wait_ctx();
   dim3 grid(a.n_tiles, h_kv);
-  score_kernel<G><<<grid, 192, smem, st>>>(tm_q, tm_k, a);
+  score_kernel<G><<<grid, kThreads, smem, st>>>(tm_q, tm_k, a);
   return launch_status(cudaGetLastError());
 }
 
