@@ -80,6 +80,24 @@ def decode_bytes(shape: synth.Shape, lens):
     return float(kc1 + kv + small)
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(dist, x: float, device) -> float:
+    """Maximum of a per-rank float over all ranks (identity without a group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job units/s: every rank processes its own replica; the step time
+    is the slowest rank's."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -177,6 +195,10 @@ def run_ours(args, rank, world, local_rank, dist):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.only == "decode":   # profiling runs: the decode steps only
+        dec = _decode(args, infv2, torch, None, rank, dev, torch.cuda.current_stream(),
+                      lambda x: x, DecodeState)
+        return {"metric": METRIC, "decode": dec}
     shape = synth.CONFIGS[args.workload]["shape"]
     n = shape.n
     p = infv2.params_of(shape)
@@ -192,12 +214,8 @@ def run_ours(args, rank, world, local_rank, dist):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x):
+        return max_over_ranks(dist, x, dev)
 
     def step():
         infv2.infv2_prefill(p, q, k, v, cu, workspace=ws, o=o, lse=lse)
@@ -221,8 +239,7 @@ def run_ours(args, rank, world, local_rank, dist):
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     clk = clocks.stop() if clocks else None
-    ms = max_over_ranks(ms)
-    pl = infv2.infv2_prefill_workspace_size(p, cu)
+    ms = max_ranks(ms)
     chunk_rows = _chunk_rows(p, n)
     n_chunks = (n + chunk_rows - 1) // chunk_rows
     launches_per_step = 1 + 2 * n_chunks + 1
@@ -233,16 +250,16 @@ def run_ours(args, rank, world, local_rank, dist):
     # ---- per-stage breakdown on the same stream (CUDA events between launches)
     stage = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows)
     # ---- end to end through host buffers
-    e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks)
+    e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_ranks)
     # ---- decode
-    dec = _decode(args, infv2, torch, shape, rank, dev, stream, max_over_ranks, DecodeState)
+    dec = _decode(args, infv2, torch, shape, rank, dev, stream, max_ranks, DecodeState)
     if infv2.infv2_device_status() != 0:
         raise RuntimeError("kernel error word set during the benchmark")
 
     work = prefill_work(shape, n)
     flops = work["score"] + work["attn"]
     peaks = measured_peaks()
-    tps = world * n / (ms / 1e3)
+    tps = job_throughput(world, n, ms)
     tflops = world * flops / (ms / 1e3) / 1e12
     # dominant kernel and its roofline
     dom = max(stage["per_kernel"], key=lambda kk: stage["per_kernel"][kk]["ms_per_step"])
@@ -404,7 +421,7 @@ def _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_ove
     h2d = qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2
     d2h = oh.numel() * 2
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    return {"value": round(world * shape.n / (ms / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(job_throughput(world, shape.n, ms), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
@@ -537,8 +554,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["c3", "c2"], default="c3",
                     help="prefill workload: c3 (131072 tokens, the reported one) or c2 (32768)")
-    ap.add_argument("--only", choices=["all", "prefill"], default="all",
-                    help="prefill: time the prefill steps only (for profiler runs)")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="prefill / decode: time only that part (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -32,6 +32,8 @@ constexpr int kHalf = 64 * 64 * 2;        // 64 keys x 64 dims of bf16 = 8 KB
 // rarely.  The final normalisation makes the result independent of it.
 constexpr float kRescaleSlack = 8.0f;
 constexpr int kStageBytes = 4 * kHalf;    // K (2 halves) + V (2 halves)
+constexpr int kQHalf = 16 * 128;          // 16 heads x 64 dims of bf16 = 2 KB
+constexpr int kQSlot = 2 * kQHalf;        // one item's Q rows
 constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -97,19 +99,26 @@ __device__ __forceinline__ void item_range(const AttnArgs& a, const Item& it, in
 __device__ __forceinline__ int block_at(const int* row, int e) { return row ? __ldg(row + e) : e; }
 
 __global__ void __launch_bounds__(160, 2)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* red_o = reinterpret_cast<float*>(base + kStages * kStageBytes);  // [4][16][128]
+  // [K/V stages][Q ring][merge buffers][barriers]; TMA destinations with the
+  // 128-byte swizzle (stages, Q ring) start on 1024-byte boundaries
+  uint8_t* qring = base + kStages * kStageBytes;                          // [2][2 halves][16][128 B]
+  float* red_o = reinterpret_cast<float*>(qring + 2 * kQSlot);            // [4][16][128]
   float* red_m = red_o + 4 * 16 * 128;                                    // [4][16]
   float* red_l = red_m + 64;                                              // [4][16]
   uint64_t* bars = reinterpret_cast<uint64_t*>(red_l + 64);
   const uint32_t stage0 = smem_u32(base);
+  const uint32_t q0 = smem_u32(qring);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kStages;
   const uint32_t cbar = empty0 + 8 * kStages;  // consumer-group barrier
+  const uint32_t qfull0 = cbar + 8;            // Q ring: 2 slots
+  const uint32_t qempty0 = qfull0 + 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -122,20 +131,36 @@ __global__ void __launch_bounds__(160, 2)
       mbar_init(empty0 + 8 * s, 4);
     }
     mbar_init(cbar, 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(qfull0 + 8 * x, 1);
+      mbar_init(qempty0 + 8 * x, 4);
+    }
     fence_mbar_init();
   }
+  // Q rows beyond the group (G < 16) are never written by TMA: keep them zero
+  for (int x = threadIdx.x; x < 2 * kQSlot / 16; x += blockDim.x)
+    reinterpret_cast<uint4*>(qring)[x] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   __syncthreads();
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      long long pc = 0;
+      long long pc = 0, qc = 0;
       bool ok = true;
-      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++qc) {
         const Item it = item_of(a, w);
         const int pos = a.decode ? __ldg(a.seqlens + it.r) : it.r;
+        {  // this item's Q rows (the G heads of group g) into the Q ring
+          const int qs = (int)(qc & 1);
+          if (!mbar_wait(qempty0 + 8 * qs, (uint32_t)((qc >> 1) & 1) ^ 1u, a.wait)) break;
+          mbar_expect_tx(qfull0 + 8 * qs, 2 * G * 128);
+          tma_load_3d(q0 + qs * kQSlot, &tm_q, qfull0 + 8 * qs, 0, it.g * G, it.r);
+          tma_load_3d(q0 + qs * kQSlot + kQHalf, &tm_q, qfull0 + 8 * qs, 64, it.g * G, it.r);
+        }
         const int* row;
         int e0, e1;
         item_range(a, it, pos, row, e0, e1);
@@ -167,6 +192,8 @@ __global__ void __launch_bounds__(160, 2)
       }
       for (long long x = pc > kStages ? pc - kStages : 0; x < pc; ++x)
         (void)mbar_wait(full0 + 8 * (int)(x % kStages), (uint32_t)((x / kStages) & 1), a.wait);
+      for (long long x = qc > 2 ? qc - 2 : 0; x < qc; ++x)
+        (void)mbar_wait(qfull0 + 8 * (int)(x & 1), (uint32_t)((x >> 1) & 1), a.wait);
     }
     return;
   }
@@ -178,21 +205,26 @@ __global__ void __launch_bounds__(160, 2)
   long long cc = 0;
   uint32_t cphase = 0;
   bool ok = true;
-  for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+  long long qc = 0;
+  for (long long w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++qc) {
     const Item it = item_of(a, w);
     const int pos = a.decode ? __ldg(a.seqlens + it.r) : it.r;  // query position
-    // Q fragments (A operand, 16 rows = heads of the group, zero beyond G)
+    // Q fragments (A operand, 16 rows = heads of the group) from the Q ring
     uint32_t qa[8][4];
     {
-      const uint16_t* qrow = a.q + ((size_t)it.r * a.h_q + (size_t)it.g * G) * 128;
+      const int qs = (int)(qc & 1);
+      if (!mbar_wait(qfull0 + 8 * qs, (uint32_t)((qc >> 1) & 1), a.wait)) break;
+      const int mi = lane >> 3, rr = lane & 7;
+      const int row = rr + ((mi & 1) << 3);  // matrices: rows 0-7 / 8-15, k 0-7 / 8-15
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const int c0 = 16 * ks + 2 * tig;
-        qa[ks][0] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + gid * 128 + c0)) : 0u;
-        qa[ks][1] = gid + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + (gid + 8) * 128 + c0)) : 0u;
-        qa[ks][2] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + gid * 128 + c0 + 8)) : 0u;
-        qa[ks][3] = gid + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + (gid + 8) * 128 + c0 + 8)) : 0u;
+        const int chunk = (ks & 3) * 2 + (mi >> 1);
+        ldsm_x4(q0 + qs * kQSlot + (ks >> 2) * kQHalf + sw_off(row, chunk), qa[ks][0], qa[ks][1],
+                qa[ks][2], qa[ks][3]);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
     }
     float o[16][4];
 #pragma unroll
@@ -202,8 +234,11 @@ __global__ void __launch_bounds__(160, 2)
     const int* row;
     int e0, e1;
     item_range(a, it, pos, row, e0, e1);
+    int chunk_b = 0;
     for (int e = e0; e < e1; ++e) {
-      const int b = block_at(row, e);
+      if (((e - e0) & 31) == 0)  // next 32 entries of the list, one per lane
+        chunk_b = e + lane < e1 ? block_at(row, e + lane) : -1;
+      const int b = __shfl_sync(0xFFFFFFFFu, chunk_b, (e - e0) & 31);
       if (b < 0) continue;
       const int s = (int)(cc % kStages);
       if (!mbar_wait(full0 + 8 * s, (uint32_t)((cc / kStages) & 1), a.wait)) {
@@ -212,19 +247,29 @@ __global__ void __launch_bounds__(160, 2)
       }
       const uint32_t kbase = stage0 + s * kStageBytes;
       const uint32_t vbase = kbase + 2 * kHalf;
-      // ---- S = Q K^T for keys kb..kb+15 (two n-tiles of 8 keys)
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // ---- S = Q K^T for keys kb..kb+15 (two n-tiles of 8 keys); the two
+      // head-dim halves accumulate separately: four independent MMA chains
+      float sc[2][4], sd[2][4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) sc[0][x] = sc[1][x] = sd[0][x] = sd[1][x] = 0.f;
       {
         const int mi = lane >> 3, rr = lane & 7;
         const int key = kb + rr + ((mi >> 1) << 3);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const int chunk = (ks & 3) * 2 + (mi & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kbase + (ks >> 2) * kHalf + sw_off(key, chunk), b0, b1, b2, b3);
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t b0, b1, b2, b3, e0, e1, e2, e3;
+          ldsm_x4(kbase + sw_off(key, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+          ldsm_x4(kbase + kHalf + sw_off(key, ks * 2 + (mi & 1)), e0, e1, e2, e3);
           mma16816(sc[0], qa[ks], b0, b1);
           mma16816(sc[1], qa[ks], b2, b3);
+          mma16816(sd[0], qa[ks + 4], e0, e1);
+          mma16816(sd[1], qa[ks + 4], e2, e3);
         }
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        sc[0][x] += sd[0][x];
+        sc[1][x] += sd[1][x];
       }
       // ---- causal mask (only a block reaching past the query) and online
       // softmax with a lazily raised reference max (rows gid and gid+8)
@@ -396,7 +441,12 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
                        cudaStream_t st) {
   const long long n_items = (long long)a.h_kv * a.n_rows * a.n_split;
   if (n_items == 0) return INFV2_OK;
-  const int smem = kStages * kStageBytes + (4 * 16 * 128 + 128) * 4 + 8 * (2 * kStages + 1) + 1024;
+  const int G = a.h_q / a.h_kv;
+  CUtensorMap tm_q;  // q [rows, h_q, 128]: one item = G heads of one row
+  if (!make_tmap_3d(&tm_q, a.q, 128, a.h_q, a.n_rows, 256, (uint64_t)a.h_q * 256, 64, G, 1))
+    return INFV2_ERR_CUDA;
+  const int smem = kStages * kStageBytes + (4 * 16 * 128 + 128) * 4 + 2 * kQSlot +
+                   8 * (2 * kStages + 1 + 4) + 1024;
   if (!set_smem(sparse_attn_kernel, smem)) return INFV2_ERR_CUDA;
   int per_sm = 1;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_attn_kernel, 160, smem) !=
@@ -404,7 +454,7 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
     per_sm = 1;
   const long long slots = (long long)per_sm * sm_count();
   const long long grid = n_items < slots ? n_items : slots;
-  sparse_attn_kernel<<<(unsigned)grid, 160, smem, st>>>(tm_k, tm_v, a);
+  sparse_attn_kernel<<<(unsigned)grid, 160, smem, st>>>(tm_q, tm_k, tm_v, a);
   return launch_status(cudaGetLastError());
 }
 

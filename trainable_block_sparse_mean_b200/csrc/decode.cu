@@ -231,25 +231,21 @@ __global__ void __launch_bounds__(256) decode_shared_kernel(const int* seqlens, 
   ws_shared[((size_t)s * h_kv + g) * ld + j] = acc;
 }
 
-// 4. selection, one warp per (sequence, kv head).
-__global__ void __launch_bounds__(256) decode_select_kernel(const int* seqlens, int batch, int h_kv,
-                                                            int cap, int n_init, int n_local, int k,
-                                                            int ld, const float* ws_shared,
-                                                            int* idx, int keys_per_warp) {
+// 4. selection, one CTA of 256 threads per (sequence, kv head).
+__global__ void __launch_bounds__(256) decode_select_kernel(const int* seqlens, int h_kv, int cap,
+                                                            int n_init, int n_local, int k, int ld,
+                                                            const float* ws_shared, int* idx,
+                                                            int n_keys) {
   extern __shared__ __align__(16) uint32_t sm_sel[];
-  const int warp = threadIdx.x >> 5;
-  const int w = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (w >= batch * h_kv) return;
-  const int s = w / h_kv, g = w % h_kv;
+  const int s = blockIdx.x / h_kv, g = blockIdx.x % h_kv;
   const int L = seqlens[s];
   int* out = idx + ((size_t)s * h_kv + g) * k;
   if (L < 0 || L >= cap) {
-    for (int x = threadIdx.x & 31; x < k; x += 32) out[x] = -1;
+    for (int x = threadIdx.x; x < k; x += blockDim.x) out[x] = -1;
     return;
   }
-  uint32_t* keys = sm_sel + (size_t)warp * (keys_per_warp + 256);
-  select_row_warp(ws_shared + ((size_t)s * h_kv + g) * ld, visible_kernels(L, 32, 16), L, n_init,
-                  n_local, k, keys, keys + keys_per_warp, out);
+  select_row_cta(ws_shared + ((size_t)s * h_kv + g) * ld, visible_kernels(L, 32, 16), L, n_init,
+                 n_local, k, sm_sel, sm_sel + n_keys, sm_sel + n_keys + 256, out);
 }
 
 // 6. merge the attention splits; advance seqlens.
@@ -348,18 +344,13 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
   {
-    const int n_blk = (cap + 63) / 64;
-    const int keys_per_warp = ((n_blk + 3) / 4) * 4;
-    const int per_warp = (keys_per_warp + 256) * 4;
-    int warps = 8;
-    while (warps > 1 && warps * per_warp > 200 * 1024) warps >>= 1;
-    if (per_warp > 200 * 1024) return INFV2_ERR_UNSUPPORTED;
-    const int smem = warps * per_warp;
+    const int n_keys = (((cap + 63) / 64 + 3) / 4) * 4;
+    const int smem = (n_keys + 256 + 4) * 4;
+    if (smem > 200 * 1024) return INFV2_ERR_UNSUPPORTED;
     if (!set_smem(decode_select_kernel, smem)) return INFV2_ERR_CUDA;
-    const int rows = batch * p->h_kv;
-    decode_select_kernel<<<(rows + warps - 1) / warps, warps * 32, smem, cs>>>(
-        seqlens, batch, p->h_kv, cap, p->n_init, p->n_local, p->k, d.ld, ws_shared, idx,
-        keys_per_warp);
+    decode_select_kernel<<<batch * p->h_kv, 256, smem, cs>>>(seqlens, p->h_kv, cap, p->n_init,
+                                                              p->n_local, p->k, d.ld, ws_shared,
+                                                              idx, n_keys);
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
   {

@@ -19,8 +19,10 @@
 //           token is a sum over G adjacent columns inside one thread, and the
 //           128 lanes store 128 consecutive floats of S^shared per token.
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps
-// 2-9 softmax / epilogue: two warpgroups, each owning 64 of a tile's 128
-// columns (pass-1 row statistics are merged through shared memory).
+// 2-17 softmax / epilogue: four warpgroups, each owning 32 of a tile's 128
+// columns (pass-1 row statistics are merged through shared memory).  A
+// quarter of the exponentials run on the FMA pipe (exp2_fma) so that the MUFU
+// unit is not the only pipe doing the softmax.
 // Accumulators are double-buffered in TMEM (2 x 128 columns) so the next
 // tile's MMA overlaps the current tile's epilogue.
 #include "common.cuh"
@@ -31,7 +33,9 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
-constexpr int kEpiWarps = 8;               // two epilogue warpgroups
+constexpr int kEpiWarps = 16;              // four epilogue warpgroups
+constexpr int kColGroups = kEpiWarps / 4;  // column groups of 128 / kColGroups columns
+constexpr int kCols = 128 / kColGroups;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -58,8 +62,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   float* s_lse2 = reinterpret_cast<float*>(base + kTileBytes * (1 + kStages));
-  float* s_part = s_lse2 + 128;  // [2 halves][128 rows][max, sum]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + 2 * 128 * 2);
+  float* s_part = s_lse2 + 128;  // [column group][128 rows][max, sum]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + kColGroups * 128 * 2);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4);
   ScoreSmem S;
   S.q = smem_u32(base);
@@ -168,9 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------- epilogue warps
     const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
-    const int half = (warp - 2) >> 2;    // columns 64*half .. +63 of every tile
+    const int cg = (warp - 2) >> 2;      // columns kCols*cg .. +kCols-1 of every tile
     const int r = quarter * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 64;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + cg * kCols;
     const int tq_r = r / G;
     const int i_r = i0 + tq_r;
     const int nv_r = i_r <= i_last ? visible_kernels(i_r, 32, 16) : 0;
@@ -181,56 +185,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = it & 1;
       if (!mbar_wait(S.acc_full + 8 * b, (it >> 1) & 1, a.wait)) break;
       tc_fence_after();
-      float v[64];
-      {
-        float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-        float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
-        tmem_ld32(lane_base + b * 128, v0);
-        tmem_ld32(lane_base + b * 128 + 32, v1);
-        tmem_ld_wait();
-      }
+      float v[32];
+      tmem_ld32(lane_base + b * 128, v);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);  // TMEM buffer free again
       if (it < n_kt) {
-        // pass 1: row r, kernels it*128 + 64*half .. +63
-        const int jb = it * 128 + half * 64;
-        if (jb + 64 > nv_r) {
+        // pass 1: row r, kernels it*128 + kCols*cg .. +31
+        const int jb = it * 128 + cg * kCols;
+        if (jb + 32 > nv_r) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
+          for (int e = 0; e < 32; ++e)
             if (jb + e >= nv_r) v[e] = -INFINITY;
         }
-        float cm = v[0];
+        float t4[4];
 #pragma unroll
-        for (int e = 1; e < 64; ++e) cm = fmaxf(cm, v[e]);
+        for (int x = 0; x < 4; ++x)
+          t4[x] = fmaxf(fmaxf(fmaxf(v[x], v[x + 4]), fmaxf(v[x + 8], v[x + 12])),
+                        fmaxf(fmaxf(v[x + 16], v[x + 20]), fmaxf(v[x + 24], v[x + 28])));
+        const float cm = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
         if (cm > vmax) {
           l *= fast_exp2((vmax - cm) * c);
           vmax = cm;
         }
         if (vmax != -INFINITY) {
           const float mneg = -vmax * c;
-          float p0 = 0.f, p1 = 0.f;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            p0 += fast_exp2(fmaf(v[e], c, mneg));
-            p1 += fast_exp2(fmaf(v[e + 1], c, mneg));
+          for (int e = 0; e < 32; ++e) {
+            const float x = fmaf(v[e], c, mneg);
+            ps[e & 3] += (e & 3) == 3 ? exp2_fma(x) : fast_exp2(x);
           }
-          l += p0 + p1;
+          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
         if (it == n_kt - 1) {
-          // merge the two column halves of row r
-          s_part[(half * 128 + r) * 2 + 0] = vmax;
-          s_part[(half * 128 + r) * 2 + 1] = l;
+          // merge the column groups' statistics of row r
+          s_part[(cg * 128 + r) * 2 + 0] = vmax;
+          s_part[(cg * 128 + r) * 2 + 1] = l;
           __syncwarp();
           if (lane == 0) mbar_arrive(S.lse_ready);
           if (!mbar_wait(S.lse_ready, 0, a.wait)) break;
-          if (half == 0) {
-            const float m0 = s_part[r * 2], l0 = s_part[r * 2 + 1];
-            const float m1 = s_part[(128 + r) * 2], l1 = s_part[(128 + r) * 2 + 1];
-            const float M = fmaxf(m0, m1);
+          if (cg == 0) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int x = 0; x < kColGroups; ++x) M = fmaxf(M, s_part[(x * 128 + r) * 2]);
             float L = 0.f;
-            if (m0 != -INFINITY) L += l0 * fast_exp2((m0 - M) * c);
-            if (m1 != -INFINITY) L += l1 * fast_exp2((m1 - M) * c);
+#pragma unroll
+            for (int x = 0; x < kColGroups; ++x) {
+              const float mx = s_part[(x * 128 + r) * 2];
+              if (mx != -INFINITY) L += s_part[(x * 128 + r) * 2 + 1] * fast_exp2((mx - M) * c);
+            }
             const float lse2 = L > 0.f ? M * c + __log2f(L) : -INFINITY;
             s_lse2[r] = lse2;
             if (a.score_lse && i_r <= i_last)
@@ -241,16 +246,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(S.lse_ready, 1, a.wait)) break;  // all 128 lse2 in smem
         }
       } else {
-        // pass 2: kernel j = (it - n_kt)*128 + r; columns 64*half.. = tokens
+        // pass 2: kernel j = (it - n_kt)*128 + r; this group's columns = tokens
         const int j = (it - n_kt) * 128 + r;
+        constexpr int TPG = kCols / G > 0 ? kCols / G : 1;  // tokens per column group
+        static_assert(G <= kCols, "a token's heads must fit in one column group");
+        const float4* lse4 = reinterpret_cast<const float4*>(s_lse2 + cg * kCols);
 #pragma unroll
-        for (int t = 0; t < 64 / G; ++t) {
-          const int tq = half * (64 / G) + t;
+        for (int t = 0; t < TPG; ++t) {
+          const int tq = cg * TPG + t;
           const int i = i0 + tq;
-          float ssum = 0.f;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+          if constexpr (G >= 4) {
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh)
-            ssum += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
+            for (int h4 = 0; h4 < G / 4; ++h4) {
+              const float4 L4 = lse4[(t * G) / 4 + h4];  // broadcast read
+              ps[0] += fast_exp2(fmaf(v[t * G + 4 * h4 + 0], c, -L4.x));
+              ps[1] += fast_exp2(fmaf(v[t * G + 4 * h4 + 1], c, -L4.y));
+              ps[2] += fast_exp2(fmaf(v[t * G + 4 * h4 + 2], c, -L4.z));
+              ps[3] += exp2_fma(fmaf(v[t * G + 4 * h4 + 3], c, -L4.w));
+            }
+          } else {
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+              ps[hh] += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
+          }
+          const float ssum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
           if (i <= i_last && j < visible_kernels(i, 32, 16))
             out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
         }
@@ -277,8 +297,8 @@ int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h
   // K^C1 map; an empty K^C1 (nc == 0) still needs a valid map, one row is enough
   if (!make_tmap_3d(&tm_k, kc1, 128, h_kv, nc > 0 ? nc : 1, 256, (uint64_t)h_kv * 256, 64, 1, 128))
     return INFV2_ERR_CUDA;
-  const int smem = kTileBytes * (1 + kStages) + 128 * 4 + 2 * 128 * 2 * 4 + 8 * (2 + 2 * kStages + 4) +
-                   16 + 1024;
+  const int smem = kTileBytes * (1 + kStages) + 128 * 4 + kColGroups * 128 * 2 * 4 +
+                   8 * (2 + 2 * kStages + 4) + 16 + 1024;
   if (!set_smem(score_kernel<G>, smem)) return INFV2_ERR_CUDA;
   ScoreArgs a;
   a.q_begin = q_begin;

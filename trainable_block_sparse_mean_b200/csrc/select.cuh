@@ -39,29 +39,40 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
     for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
     return;
   }
-  // ---- max pooling into order keys (forced blocks get the top key)
+  // ---- max pooling into order keys (forced blocks get the top key); four
+  // 512-byte row segments are loaded before any is used
   float carry = -INFINITY;  // S^shared[4*base - 1] for the next chunk's lane 0
-  for (int base = 0; base < n_cand; base += 32) {
-    const int b = base + lane;
-    float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    const int j0 = 4 * b;
-    if (b < n_cand) {
-      if (j0 + 3 < nv) {
-        v = *reinterpret_cast<const float4*>(row + j0);
-      } else {
-        if (j0 + 0 < nv) v.x = row[j0 + 0];
-        if (j0 + 1 < nv) v.y = row[j0 + 1];
-        if (j0 + 2 < nv) v.z = row[j0 + 2];
+  for (int base0 = 0; base0 < n_cand; base0 += 128) {
+    float4 vv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = base0 + 32 * u + lane;
+      const int j0 = 4 * b;
+      float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (b < n_cand) {
+        if (j0 + 3 < nv) {
+          v = __ldg(reinterpret_cast<const float4*>(row + j0));
+        } else {
+          if (j0 + 0 < nv) v.x = row[j0 + 0];
+          if (j0 + 1 < nv) v.y = row[j0 + 1];
+          if (j0 + 2 < nv) v.z = row[j0 + 2];
+        }
       }
+      vv[u] = v;
     }
-    // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
-    float prev = __shfl_up_sync(0xFFFFFFFFu, v.w, 1);
-    if (lane == 0) prev = carry;
-    carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
-    if (b < n_cand) {
-      const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
-      const bool forced = b < n_init || b > bi - n_local;
-      keys[b] = forced ? kForcedKey : float_key(m);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = base0 + 32 * u + lane;
+      const float4 v = vv[u];
+      // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
+      float prev = __shfl_up_sync(0xFFFFFFFFu, v.w, 1);
+      if (lane == 0) prev = carry;
+      carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
+      if (b < n_cand) {
+        const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
+        const bool forced = b < n_init || b > bi - n_local;
+        keys[b] = forced ? kForcedKey : float_key(m);
+      }
     }
   }
   __syncwarp();
@@ -132,6 +143,99 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
   }
   for (int x = written + lane; x < k; x += 32) out[x] = -1;
   __syncwarp();
+}
+
+// Same selection for one row with a whole CTA of 256 threads (used when there
+// are few rows, e.g. one per sequence in decode).  `keys` holds >= bi+1 words,
+// `hist` 256 words and `bcast` 4 words, all in shared memory.
+__device__ __forceinline__ void select_row_cta(const float* __restrict__ row, int nv, int i,
+                                               int n_init, int n_local, int k, uint32_t* keys,
+                                               uint32_t* hist, uint32_t* bcast,
+                                               int* __restrict__ out) {
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
+  const int bi = i >> 6;
+  const int n_cand = bi + 1;
+  if (n_cand <= k) {
+    for (int b = t; b < k; b += blockDim.x) out[b] = b < n_cand ? b : -1;
+    return;
+  }
+  for (int b = t; b < n_cand; b += blockDim.x) {
+    const int j0 = 4 * b;
+    float m = -INFINITY;
+    if (j0 - 1 >= 0 && j0 - 1 < nv) m = row[j0 - 1];
+    if (j0 + 3 < nv) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + j0));
+      m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    } else {
+      for (int e = 0; e < 3; ++e)
+        if (j0 + e < nv) m = fmaxf(m, row[j0 + e]);
+    }
+    const bool forced = b < n_init || b > bi - n_local;
+    keys[b] = forced ? kForcedKey : float_key(m);
+  }
+  __syncthreads();
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int x = t; x < 256; x += blockDim.x) hist[x] = 0;
+    __syncthreads();
+    for (int b = t; b < n_cand; b += blockDim.x) {
+      const uint32_t key = keys[b];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t cnt[8];
+      uint32_t local = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt[e] = hist[255 - 8 * lane - e];
+        local += cnt[e];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      const uint32_t before = incl - local;
+      if (before < (uint32_t)remaining && (uint32_t)remaining <= incl) {
+        uint32_t run = before;
+        for (int e = 0; e < 8; ++e) {
+          if (run + cnt[e] >= (uint32_t)remaining) {
+            bcast[0] = 255u - 8u * lane - e;
+            bcast[1] = run;
+            break;
+          }
+          run += cnt[e];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= bcast[0] << shift;
+    pmask |= 255u << shift;
+    remaining -= (int)bcast[1];
+    __syncthreads();
+  }
+  if (warp == 0) {
+    const uint32_t T = prefix;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int eq_seen = 0, written = 0;
+    for (int base = 0; base < n_cand; base += 32) {
+      const int b = base + lane;
+      const uint32_t key = b < n_cand ? keys[b] : 0u;
+      const bool eq = b < n_cand && key == T;
+      const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
+      const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
+      eq_seen += __popc(eqb);
+      const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
+      if (sel) out[written + __popc(selb & lt_mask)] = b;
+      written += __popc(selb);
+    }
+    for (int x = written + lane; x < k; x += 32) out[x] = -1;
+  }
 }
 
 }  // namespace infv2
