@@ -430,7 +430,9 @@ def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, Decod
     split-KV attention, combine: 7 launches) is captured once into a CUDA graph,
     as a serving loop would run it, and the graphs are replayed in order (each
     replay appends its own token and advances seqlens on the device)."""
-    cfg = synth.CONFIGS["c4"]
+    cfg = dict(synth.CONFIGS["c4"])
+    if args.decode_small:   # profiler runs: 8 sequences of at most 32k tokens
+        cfg.update(batch=8, len_lo=16384, len_hi=32768)
     sh = cfg["shape"]
     steps_avail = cfg["steps"]
     data = synth.make_decode(sh, cfg["batch"], cfg["len_lo"], cfg["len_hi"], steps_avail,
@@ -554,6 +556,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["c3", "c2"], default="c3",
                     help="prefill workload: c3 (131072 tokens, the reported one) or c2 (32768)")
+    ap.add_argument("--decode-small", action="store_true",
+                    help="with --only decode: 8 sequences of 16k-32k tokens (profiler runs)")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="prefill / decode: time only that part (for profiler runs)")
     args = ap.parse_args()

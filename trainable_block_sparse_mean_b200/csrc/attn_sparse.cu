@@ -31,6 +31,7 @@ constexpr int kHalf = 64 * 64 * 2;        // 64 keys x 64 dims of bf16 = 8 KB
 // than this (log2 units): probabilities stay below 2^8, and O, l are rescaled
 // rarely.  The final normalisation makes the result independent of it.
 constexpr float kRescaleSlack = 8.0f;
+constexpr int kMaxSplit = 16;             // most pieces a split row may have
 constexpr int kStageBytes = 4 * kHalf;    // K (2 halves) + V (2 halves)
 constexpr int kQHalf = 16 * 128;          // 16 heads x 64 dims of bf16 = 2 KB
 constexpr int kQSlot = 2 * kQHalf;        // one item's Q rows
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(160, 2)
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_last;  // split mode: this CTA merges the pieces of its (row, kv head)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   // [K/V stages][Q ring][merge buffers][barriers]; TMA destinations with the
@@ -427,11 +429,85 @@ __global__ void __launch_bounds__(160, 2)
           }
         }
       }
+      if (a.split_out) __threadfence();  // this piece is visible before it is counted
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(cbar);
     if (!mbar_wait(cbar, cphase & 1u, a.wait)) break;
     ++cphase;
+    if (a.split_out) {
+      // the last piece of (row, kv head) to finish merges all pieces
+      if (threadIdx.x == 0) s_last = atomicAdd(&a.counters[(size_t)it.r * a.h_kv + it.g], 1) == a.n_split - 1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(cbar);
+      if (!mbar_wait(cbar, cphase & 1u, a.wait)) break;
+      ++cphase;
+      if (s_last) {
+        __threadfence();
+        const int t = threadIdx.x;
+        const int rowh = t >> 3;
+        const int d0 = (t & 7) * 16;
+        if (rowh < G) {
+          const int h = it.g * G + rowh;
+          const size_t slot0 = ((size_t)it.r * a.h_q + h) * a.n_split;
+          // all pieces' (max, sum) first, independent loads in flight
+          float2 mlv[kMaxSplit];
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplit; ++sp)
+            mlv[sp] = sp < a.n_split
+                          ? __ldcg(reinterpret_cast<const float2*>(a.part_ml + (slot0 + sp) * 2))
+                          : make_float2(-INFINITY, 0.f);
+          float M = -INFINITY;
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplit; ++sp) M = fmaxf(M, mlv[sp].x);
+          float L = 0.f, acc[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) acc[x] = 0.f;
+          if (M != -INFINITY) {
+#pragma unroll 4
+            for (int sp = 0; sp < kMaxSplit; ++sp) {
+              if (sp >= a.n_split) break;
+              const float sc = mlv[sp].x == -INFINITY ? 0.f : fast_exp2(mlv[sp].x - M);
+              L += mlv[sp].y * sc;
+              const float4* src = reinterpret_cast<const float4*>(a.part_o + (slot0 + sp) * 128 + d0);
+              const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1), v2 = __ldcg(src + 2),
+                           v3 = __ldcg(src + 3);
+              const float4 vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                acc[4 * x + 0] += vv[x].x * sc;
+                acc[4 * x + 1] += vv[x].y * sc;
+                acc[4 * x + 2] += vv[x].z * sc;
+                acc[4 * x + 3] += vv[x].w * sc;
+              }
+            }
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          uint4 w0, w1;
+          w0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+          w0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+          w0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+          w0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+          w1.x = pack_bf16(acc[8] * inv, acc[9] * inv);
+          w1.y = pack_bf16(acc[10] * inv, acc[11] * inv);
+          w1.z = pack_bf16(acc[12] * inv, acc[13] * inv);
+          w1.w = pack_bf16(acc[14] * inv, acc[15] * inv);
+          uint16_t* dst = a.o + ((size_t)it.r * a.h_q + h) * 128 + d0;
+          reinterpret_cast<uint4*>(dst)[0] = w0;
+          reinterpret_cast<uint4*>(dst)[1] = w1;
+          if (a.lse && (t & 7) == 0)
+            a.lse[(size_t)it.r * a.h_q + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+        }
+        if (t == 0) {
+          a.counters[(size_t)it.r * a.h_kv + it.g] = 0;
+          int* seq_done = a.counters + (size_t)a.n_rows * a.h_kv + it.r;
+          if (atomicAdd(seq_done, 1) == a.h_kv - 1) {  // every kv head of this row merged
+            *seq_done = 0;
+            if (a.decode && pos >= 0 && pos < a.cap) a.seqlens_out[it.r] = pos + 1;
+          }
+        }
+      }
+    }
   }
 }
 

@@ -13,6 +13,7 @@ struct AttnArgs {
   float scale_log2;        // scale * log2(e)
   int decode;              // 1: K/V in cache layout, query position = seqlens[row]
   const int* seqlens;
+  int* seqlens_out;        // decode split mode: advanced once all of a row is merged
   int n_split, blocks_per_split;  // the block list is cut into n_split pieces
   int split_out;           // 1: write partials (part_o, part_ml) instead of o / lse
   uint16_t* o;             // o + (row*h_q + h)*128
@@ -20,6 +21,9 @@ struct AttnArgs {
   long long lse_ld;
   float* part_o;           // [row][h_q][n_split][128] unnormalised sums
   float* part_ml;          // [row][h_q][n_split][2]   (max in log2 units, sum)
+  int* counters;           // split mode: [rows * h_kv] pieces done, then [rows] heads done;
+                           // the last piece merges and (last head) advances seqlens
+  int cap;                 // decode: cache capacity (a position >= cap is not advanced)
   WaitCtx wait;
 };
 

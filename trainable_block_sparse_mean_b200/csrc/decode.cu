@@ -2,18 +2,21 @@
 //
 // MiniCPM4 "InfLLM v2" blog (query/key granularity): selection is per query
 // token, so a decoding token selects its own blocks and attends to at most k*B
-// keys.  The step is memory-bound (it reads K^C1 and the selected K/V once), so
-// it is split over many CTAs:
-//   1. append     write the new K/V row; if it completes a stage-1 kernel,
-//                 write that K^C1 row (same fp64 mean as prefill compression)
-//   2. logits     z = scale*log2(e) * q.K^C1 for all visible kernels, split in
-//                 chunks of 256 kernels, plus each chunk's per-head (max, sum)
-//   3. shared     per-head lse from the chunk partials, then
-//                 S^shared[j] = sum_h exp2(z_hj - lse_h)
-//   4. select     max pooling + top-k, one warp per (sequence, kv head)
-//   5. attention  the block-sparse kernel over the selected blocks, with the
-//                 block list split so that several CTAs share one sequence
-//   6. combine    merge the splits, write O / lse, advance seqlens.
+// keys.  The step is memory-bound (it reads K^C1 and the selected K/V once) and
+// runs as three kernels:
+//   1. logits     (one CTA per 256 kernels of a (sequence, kv head)): the CTA
+//                 of chunk 0 appends the new K/V row to the cache; the CTA whose
+//                 chunk holds a kernel completed by the new token writes that
+//                 K^C1 row (same fp64 mean as prefill compression); every CTA
+//                 computes z = scale*log2(e) * q.K^C1 for its visible kernels
+//                 (stored head-minor) and each head's (max, sum) over the chunk
+//   2. select     (one CTA per (sequence, kv head)): per-head lse from the chunk
+//                 partials, S^shared[j] = sum_h exp2(z_hj - lse_h) for the
+//                 kernels of each block, max pooling and the radix top-k
+//   3. attention  the block-sparse kernel over the selected blocks, the list
+//                 split into pieces of 8 blocks so that several CTAs share a
+//                 sequence; the last piece to finish merges the pieces, writes
+//                 O / lse and, for the last kv head, advances seqlens.
 #include "attn_sparse.cuh"
 #include "internal.cuh"
 #include "kc1_mean.cuh"
@@ -22,146 +25,156 @@
 namespace infv2 {
 namespace {
 
-constexpr int kChunk = 256;        // kernels per logits CTA
-constexpr int kBlocksPerSplit = 8; // selected blocks per attention CTA
-constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kChunk = 256;         // kernels per logits CTA
+constexpr int kBlocksPerSplit = 8;  // selected blocks per attention CTA (at least)
+constexpr int kMaxPieces = 16;      // pieces the attention kernel's merge accepts
 
 struct DecodePlan {
-  int cap_c1, zld, n_chunks, ld, n_split, G;
-  size_t off_z, off_ml, off_shared, off_idx, off_po, off_pml, total;
+  int cap_c1, n_chunks, n_split, bps, G;
+  size_t off_z, off_ml, off_idx, off_po, off_pml, off_cnt, total;
 };
 
 DecodePlan plan_decode(const infv2_params* p, int batch, int cap) {
   DecodePlan d{};
   d.G = p->h_q / p->h_kv;
   d.cap_c1 = infv2_num_kernels(p, cap);
-  d.zld = ((d.cap_c1 + 3) / 4) * 4;  // logits row pitch: 16-byte aligned rows
   d.n_chunks = (d.cap_c1 + kChunk - 1) / kChunk;
-  d.ld = shared_ld(cap);
-  d.n_split = (p->k + kBlocksPerSplit - 1) / kBlocksPerSplit;
+  d.bps = (p->k + kMaxPieces - 1) / kMaxPieces;
+  if (d.bps < kBlocksPerSplit) d.bps = kBlocksPerSplit;
+  d.n_split = (p->k + d.bps - 1) / d.bps;
   size_t off = 0;
-  d.off_z = off;
-  off += round256((size_t)batch * p->h_kv * d.G * (d.zld > 0 ? d.zld : 4) * 4);
-  d.off_ml = off;
-  off += round256((size_t)batch * p->h_kv * (d.n_chunks > 0 ? d.n_chunks : 1) * d.G * 2 * 4);
-  d.off_shared = off;
-  off += round256((size_t)batch * p->h_kv * d.ld * 4);
+  d.off_z = off;  // [batch][h_kv][cap_c1][16] logits, heads padded to 16
+  off += round256((size_t)batch * p->h_kv * (d.cap_c1 > 0 ? d.cap_c1 : 1) * 16 * 4);
+  d.off_ml = off;  // [batch][h_kv][n_chunks][16][max, sum]
+  off += round256((size_t)batch * p->h_kv * (d.n_chunks > 0 ? d.n_chunks : 1) * 16 * 2 * 4);
   d.off_idx = off;
   off += round256((size_t)batch * p->h_kv * p->k * 4);
   d.off_po = off;
   off += round256((size_t)batch * p->h_q * d.n_split * 128 * 4);
   d.off_pml = off;
   off += round256((size_t)batch * p->h_q * d.n_split * 2 * 4);
+  d.off_cnt = off;  // split counters [batch][h_kv], sequence counters [batch]
+  off += round256((size_t)batch * (p->h_kv + 1) * 4);
   d.total = off;
   return d;
 }
 
-// 1. append the new token and, if it completes a kernel, its K^C1 row.
-__global__ void __launch_bounds__(128) decode_append_kernel(
-    const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new, uint16_t* k_cache,
-    uint16_t* v_cache, uint16_t* kc1_cache, const int* seqlens, int h_kv, int cap, int cap_c1,
-    int* err) {
-  const int s = blockIdx.x;
-  const int L = seqlens[s];
-  if (L < 0 || L >= cap) {
-    if (threadIdx.x == 0) report_error(err, INFV2_ERR_INVALID_ARG);
-    return;
-  }
-  // copy: h_kv rows of 256 B for K and for V, 16 B per thread step
-  const int n16 = h_kv * 16;
-  for (int x = threadIdx.x; x < 2 * n16; x += blockDim.x) {
-    const int which = x / n16;  // 0: K, 1: V
-    const int y = x % n16;
-    const int g = y / 16, c = y % 16;
-    const uint16_t* src = (which ? v_new : k_new) + ((size_t)s * h_kv + g) * 128 + c * 8;
-    uint16_t* dst = (which ? v_cache : k_cache) + (((size_t)s * h_kv + g) * cap + L) * 128 + c * 8;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-  }
-  const int Lp = L + 1;  // length after the append
-  if (Lp >= 32 && (Lp - 32) % 16 == 0) {
-    const int j = (Lp - 32) / 16;
-    for (int y = threadIdx.x; y < n16; y += blockDim.x) {
-      const int g = y / 16, c = y % 16;
-      const uint16_t* rows = k_cache + (((size_t)s * h_kv + g) * cap + 16 * j) * 128 + c * 8;
-      const uint16_t* knew = k_new + ((size_t)s * h_kv + g) * 128 + c * 8;
-      const uint4 m = kc1_mean_slice(rows, 128, knew, L - 16 * j);
-      *reinterpret_cast<uint4*>(kc1_cache + (((size_t)s * h_kv + g) * cap_c1 + j) * 128 + c * 8) = m;
-    }
-  }
-}
-
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 2. logits for 256 kernels of one (sequence, kv head): 4 warps x 64 kernels,
-// 16 heads x 8 kernels per m16n8k16 tile, K^C1 fragments read straight from
-// global memory (each row segment is used once).
-__global__ void __launch_bounds__(128) decode_logits_kernel(
-    const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc1_cache, const int* seqlens,
-    int h_q, int h_kv, int cap, int cap_c1, int zld, int n_chunks, float scale_log2, float* ws_z,
-    float* ws_ml) {
+struct LogitsArgs {
+  const uint16_t* q;      // [batch, h_q, 128]
+  const uint16_t* k_new;  // [batch, h_kv, 128]
+  const uint16_t* v_new;
+  uint16_t* k_cache;      // [batch, h_kv, cap, 128]
+  uint16_t* v_cache;
+  uint16_t* kc1_cache;    // [batch, h_kv, cap_c1, 128]
+  const int* seqlens;
+  int h_q, h_kv, cap, cap_c1, n_chunks;
+  float scale_log2;
+  float* z;               // [batch, h_kv, cap_c1, 16]
+  float* ml;              // [batch, h_kv, n_chunks, 16, 2]
+  int* counters;          // [batch * h_kv] then [batch]
+  int* err;
+};
+
+// 1. append + incremental K^C1 + logits for 256 kernels of one (sequence, kv
+// head).  The MMA contracts over the head dim in a permuted order (both
+// operands alike) so that every lane loads 16 contiguous bytes per row: for
+// k-steps 2c and 2c+1 lane (gid, tig) holds dims 32c + 8tig .. 32c + 8tig + 7.
+__global__ void __launch_bounds__(128) decode_logits_kernel(LogitsArgs a) {
   const int chunk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-  const int L = seqlens[s];
-  if (L < 0 || L >= cap) return;
-  const int nv = visible_kernels(L, 32, 16);
+  const int t = threadIdx.x;
+  const int L = a.seqlens[s];
+  if (L < 0 || L >= a.cap) {
+    if (chunk == 0 && g == 0 && t == 0) report_error(a.err, INFV2_ERR_INVALID_ARG);
+    return;
+  }
+  const size_t sg = (size_t)s * a.h_kv + g;
+  if (chunk == 0) {
+    // append the new token's K and V rows of this kv head; reset the
+    // attention kernel's completion counters of this step
+    if (t < 32) {
+      const uint16_t* src = (t < 16 ? a.k_new : a.v_new) + sg * 128 + (t & 15) * 8;
+      uint16_t* dst = (t < 16 ? a.k_cache : a.v_cache) + (sg * a.cap + L) * 128 + (t & 15) * 8;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    }
+    if (t == 32) {
+      a.counters[sg] = 0;
+      if (g == 0) a.counters[(size_t)gridDim.z * a.h_kv + s] = 0;
+    }
+  }
+  const int nv = visible_kernels(L, 32, 16);  // includes a kernel completed by token L
   const int j_chunk = chunk * kChunk;
   if (j_chunk >= nv) return;
-  const int G = h_q / h_kv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Lp = L + 1;
+  const int j_new = (Lp >= 32 && (Lp - 32) % 16 == 0) ? (Lp - 32) / 16 : -1;
+  if (j_new >= j_chunk && j_new < j_chunk + kChunk) {  // uniform over the CTA
+    if (t < 16) {
+      const uint16_t* rows = a.k_cache + (sg * a.cap + 16 * j_new) * 128 + t * 8;
+      const uint16_t* knew = a.k_new + sg * 128 + t * 8;
+      const uint4 m = kc1_mean_slice(rows, 128, knew, L - 16 * j_new);
+      *reinterpret_cast<uint4*>(a.kc1_cache + (sg * a.cap_c1 + j_new) * 128 + t * 8) = m;
+    }
+    __syncthreads();  // the new K^C1 row is read below by other threads
+  }
+  const int G = a.h_q / a.h_kv;
+  const int warp = t >> 5, lane = t & 31;
   const int gid = lane >> 2, tig = lane & 3;
   __shared__ float sm_m[4][16], sm_l[4][16];
 
-  uint32_t qa[8][4];
-  const uint16_t* qrow = q + ((size_t)s * h_q + (size_t)g * G) * 128;
+  // Q fragments in the permuted head-dim order
+  uint4 q0[4], q1[4];
+  {
+    const uint16_t* qrow = a.q + ((size_t)s * a.h_q + (size_t)g * G) * 128 + 8 * tig;
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const int c0 = 16 * ks + 2 * tig;
-    qa[ks][0] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + gid * 128 + c0)) : 0u;
-    qa[ks][1] = gid + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + (gid + 8) * 128 + c0)) : 0u;
-    qa[ks][2] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + gid * 128 + c0 + 8)) : 0u;
-    qa[ks][3] = gid + 8 < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + (gid + 8) * 128 + c0 + 8)) : 0u;
+    for (int c = 0; c < 4; ++c) {
+      q0[c] = gid < G ? __ldg(reinterpret_cast<const uint4*>(qrow + gid * 128 + 32 * c))
+                      : make_uint4(0u, 0u, 0u, 0u);
+      q1[c] = gid + 8 < G ? __ldg(reinterpret_cast<const uint4*>(qrow + (gid + 8) * 128 + 32 * c))
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
-  const uint16_t* kbase = kc1_cache + ((size_t)s * h_kv + g) * cap_c1 * 128;
-  float* zrow = ws_z + ((size_t)s * h_kv + g) * G * zld;
+  const uint16_t* kbase = a.kc1_cache + sg * a.cap_c1 * 128 + 8 * tig;
+  float* zbase = a.z + sg * a.cap_c1 * 16;
   float mx0 = -INFINITY, mx1 = -INFINITY;
   float zv[8][4];
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     const int jn = j_chunk + warp * 64 + nt * 8;  // first kernel of this n-tile
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int jr = jn + gid;  // kernel row this lane feeds as B
-    const bool rv = jr < nv;
-    const uint16_t* kr = kbase + (size_t)(rv ? jr : 0) * 128;
+    const int jr = jn + gid;                      // kernel row this lane loads
+    uint4 kv[4];
+    if (jr < nv) {
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t b0 = rv ? __ldg(reinterpret_cast<const uint32_t*>(kr + 16 * ks + 2 * tig)) : 0u;
-      const uint32_t b1 = rv ? __ldg(reinterpret_cast<const uint32_t*>(kr + 16 * ks + 8 + 2 * tig)) : 0u;
-      mma16816(acc, qa[ks], b0, b1);
+      for (int c = 0; c < 4; ++c)  // L2-only loads: this kernel may have written the row
+        kv[c] = __ldcg(reinterpret_cast<const uint4*>(kbase + (size_t)jr * 128 + 32 * c));
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kv[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      mma16816(acc, q0[c].x, q1[c].x, q0[c].y, q1[c].y, kv[c].x, kv[c].y);
+      mma16816(acc, q0[c].z, q1[c].z, q0[c].w, q1[c].w, kv[c].z, kv[c].w);
     }
     // acc: (head gid, kernels jn+2tig, +1), (head gid+8, same kernels)
     const int j0 = jn + 2 * tig;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = j0 + (e & 1);
-      zv[nt][e] = j < nv ? acc[e] * scale_log2 : -INFINITY;
-    }
+    for (int e = 0; e < 4; ++e) zv[nt][e] = (j0 + (e & 1)) < nv ? acc[e] * a.scale_log2 : -INFINITY;
     mx0 = fmaxf(mx0, fmaxf(zv[nt][0], zv[nt][1]));
     mx1 = fmaxf(mx1, fmaxf(zv[nt][2], zv[nt][3]));
-    if (j0 < nv) {
-      if (gid < G) {
-        if (j0 + 1 < nv) *reinterpret_cast<float2*>(zrow + (size_t)gid * zld + j0) = make_float2(zv[nt][0], zv[nt][1]);
-        else zrow[(size_t)gid * zld + j0] = zv[nt][0];
-      }
-      if (gid + 8 < G) {
-        if (j0 + 1 < nv) *reinterpret_cast<float2*>(zrow + (size_t)(gid + 8) * zld + j0) = make_float2(zv[nt][2], zv[nt][3]);
-        else zrow[(size_t)(gid + 8) * zld + j0] = zv[nt][2];
-      }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + (e & 1);
+      const int h = gid + ((e >> 1) << 3);
+      if (j < nv && h < G) zbase[(size_t)j * 16 + h] = zv[nt][e];
     }
   }
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
@@ -186,106 +199,114 @@ __global__ void __launch_bounds__(128) decode_logits_kernel(
     sm_l[warp][gid + 8] = l1;
   }
   __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
+  if (t < G) {
     float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w][h]);
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w][t]);
     float Ls = 0.f;
     for (int w = 0; w < 4; ++w)
-      if (sm_m[w][h] != -INFINITY) Ls += sm_l[w][h] * fast_exp2(sm_m[w][h] - M);
-    float* ml = ws_ml + ((((size_t)s * h_kv + g) * n_chunks + chunk) * G + h) * 2;
+      if (sm_m[w][t] != -INFINITY) Ls += sm_l[w][t] * fast_exp2(sm_m[w][t] - M);
+    float* ml = a.ml + ((sg * a.n_chunks + chunk) * 16 + t) * 2;
     ml[0] = M;
     ml[1] = Ls;
   }
 }
 
-// 3. S^shared for 256 kernels of one (sequence, kv head).
-__global__ void __launch_bounds__(256) decode_shared_kernel(const int* seqlens, int h_kv, int G,
-                                                            int cap, int zld, int n_chunks,
-                                                            int ld, const float* ws_z,
-                                                            const float* ws_ml, float* ws_shared) {
-  const int chunk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-  const int L = seqlens[s];
-  if (L < 0 || L >= cap) return;
-  const int nv = visible_kernels(L, 32, 16);
-  if (chunk * kChunk >= nv) return;
-  __shared__ float lse2[16];
-  const int used = (nv + kChunk - 1) / kChunk;
-  if (threadIdx.x < G) {
-    const float* ml = ws_ml + ((size_t)s * h_kv + g) * n_chunks * G * 2;
-    float M = -INFINITY;
-    for (int c = 0; c < used; ++c) M = fmaxf(M, ml[(c * G + threadIdx.x) * 2]);
-    float Ls = 0.f;
-    for (int c = 0; c < used; ++c) {
-      const float m = ml[(c * G + threadIdx.x) * 2];
-      if (m != -INFINITY) Ls += ml[(c * G + threadIdx.x) * 2 + 1] * fast_exp2(m - M);
-    }
-    lse2[threadIdx.x] = M + __log2f(Ls);
-  }
-  __syncthreads();
-  const int j = chunk * kChunk + threadIdx.x;
-  if (j >= nv) return;
-  const float* zrow = ws_z + ((size_t)s * h_kv + g) * G * zld;
-  float acc = 0.f;
-  for (int h = 0; h < G; ++h) acc += fast_exp2(zrow[(size_t)h * zld + j] - lse2[h]);
-  ws_shared[((size_t)s * h_kv + g) * ld + j] = acc;
-}
+struct SelectDecArgs {
+  const int* seqlens;
+  int h_kv, G, cap, cap_c1, n_chunks;
+  int n_init, n_local, k;
+  const float* z;
+  const float* ml;
+  int* idx;  // [batch, h_kv, k]
+  int n_keys;
+};
 
-// 4. selection, one CTA of 256 threads per (sequence, kv head).
-__global__ void __launch_bounds__(256) decode_select_kernel(const int* seqlens, int h_kv, int cap,
-                                                            int n_init, int n_local, int k, int ld,
-                                                            const float* ws_shared, int* idx,
-                                                            int n_keys) {
+// 2. per-head lse, S^shared per block window, max pooling and top-k for one
+// (sequence, kv head), by a CTA of 256 threads.
+__global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
   extern __shared__ __align__(16) uint32_t sm_sel[];
-  const int s = blockIdx.x / h_kv, g = blockIdx.x % h_kv;
-  const int L = seqlens[s];
-  int* out = idx + ((size_t)s * h_kv + g) * k;
-  if (L < 0 || L >= cap) {
-    for (int x = threadIdx.x; x < k; x += blockDim.x) out[x] = -1;
+  uint32_t* keys = sm_sel;
+  uint32_t* hist = keys + a.n_keys;
+  uint32_t* bcast = hist + 256;
+  float* lse2 = reinterpret_cast<float*>(bcast + 4);  // [16]
+  float* shared_s = lse2 + 16;                        // [cap_c1] S^shared of the row
+  const int sgi = blockIdx.x;
+  const int s = sgi / a.h_kv;
+  const int t = threadIdx.x;
+  const int L = a.seqlens[s];
+  int* out = a.idx + (size_t)sgi * a.k;
+  if (L < 0 || L >= a.cap) {
+    for (int x = t; x < a.k; x += blockDim.x) out[x] = -1;
     return;
   }
-  select_row_cta(ws_shared + ((size_t)s * h_kv + g) * ld, visible_kernels(L, 32, 16), L, n_init,
-                 n_local, k, sm_sel, sm_sel + n_keys, sm_sel + n_keys + 256, out);
-}
-
-// 6. merge the attention splits; advance seqlens.
-__global__ void __launch_bounds__(256) decode_combine_kernel(int* seqlens, int h_q, int cap,
-                                                             int n_split, const float* part_o,
-                                                             const float* part_ml, uint16_t* o,
-                                                             float* lse) {
-  const int s = blockIdx.x;
-  const int L = seqlens[s];
-  const bool valid = L >= 0 && L < cap;
-  for (int x = threadIdx.x; x < h_q * 32; x += blockDim.x) {
-    const int h = x / 32, d0 = (x % 32) * 4;
-    const size_t slot0 = ((size_t)s * h_q + h) * n_split;
+  const int bi = L >> 6;
+  const int n_cand = bi + 1;
+  if (n_cand <= a.k) {  // every visible block
+    for (int b = t; b < a.k; b += blockDim.x) out[b] = b < n_cand ? b : -1;
+    return;
+  }
+  const int nv = visible_kernels(L, 32, 16);
+  const int used = (nv + kChunk - 1) / kChunk;
+  {  // lse of each head over the chunk partials: 16 threads per head
+    const int h = t >> 4, c0 = t & 15;
+    const float* ml = a.ml + (size_t)sgi * a.n_chunks * 32 + h * 2;
     float M = -INFINITY;
-    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, valid ? part_ml[(slot0 + sp) * 2] : -INFINITY);
-    float Ls = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (M != -INFINITY) {
-      for (int sp = 0; sp < n_split; ++sp) {
-        const float m = part_ml[(slot0 + sp) * 2];
-        if (m == -INFINITY) continue;
-        const float sc = fast_exp2(m - M);
-        Ls += part_ml[(slot0 + sp) * 2 + 1] * sc;
-        const float4 v = *reinterpret_cast<const float4*>(part_o + (slot0 + sp) * 128 + d0);
-        acc[0] += v.x * sc;
-        acc[1] += v.y * sc;
-        acc[2] += v.z * sc;
-        acc[3] += v.w * sc;
-      }
+    for (int c = c0; c < used; c += 16) M = fmaxf(M, ml[c * 32]);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    float S = 0.f;
+    for (int c = c0; c < used; c += 16) {
+      const float m = ml[c * 32];
+      if (m != -INFINITY) S += ml[c * 32 + 1] * fast_exp2(m - M);
     }
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-    uint2 wv;
-    wv.x = *reinterpret_cast<uint32_t*>(&a0);
-    wv.y = *reinterpret_cast<uint32_t*>(&a1);
-    *reinterpret_cast<uint2*>(o + ((size_t)s * h_q + h) * 128 + d0) = wv;
-    if (lse && d0 == 0) lse[(size_t)s * h_q + h] = Ls > 0.f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) S += __shfl_xor_sync(0xFFFFFFFFu, S, o);
+    if (c0 == 0) lse2[h] = M + __log2f(S);
   }
   __syncthreads();
-  if (threadIdx.x == 0 && valid) seqlens[s] = L + 1;
+  float lse_r[16];
+#pragma unroll
+  for (int h = 0; h < 16; ++h) lse_r[h] = lse2[h];
+  // S^shared of every visible kernel into shared memory; each thread keeps
+  // the logit loads of four kernels in flight
+  const float* zrow = a.z + (size_t)sgi * a.cap_c1 * 16;
+  const int G = a.G;
+  for (int j0 = t; j0 < nv; j0 += 4 * blockDim.x) {
+    float4 v[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * blockDim.x;
+      const float4* zr = reinterpret_cast<const float4*>(zrow + (size_t)(j < nv ? j : 0) * 16);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        v[u][q4] = 4 * q4 < G ? __ldg(zr + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * blockDim.x;
+      float sh = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float vv[4] = {v[u][q4].x, v[u][q4].y, v[u][q4].z, v[u][q4].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * q4 + e < G) sh += fast_exp2(vv[e] - lse_r[4 * q4 + e]);
+      }
+      if (j < nv) shared_s[j] = sh;
+    }
+  }
+  __syncthreads();
+  // max pooling over the kernels intersecting each block (4b-1 .. 4b+3)
+  for (int b = t; b < n_cand; b += blockDim.x) {
+    const bool forced = b < a.n_init || b > bi - a.n_local;
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 4 * b - 1; j <= 4 * b + 3; ++j)
+      if (j >= 0 && j < nv) m = fmaxf(m, shared_s[j]);
+    keys[b] = forced ? kForcedKey : float_key(m);
+  }
+  __syncthreads();
+  select_topk_cta(keys, n_cand, a.k, hist, bcast, out);
 }
 
 }  // namespace
@@ -319,38 +340,54 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* ws_z = reinterpret_cast<float*>(ws + d.off_z);
   float* ws_ml = reinterpret_cast<float*>(ws + d.off_ml);
-  float* ws_shared = reinterpret_cast<float*>(ws + d.off_shared);
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(ws + d.off_idx);
-  float* part_o = reinterpret_cast<float*>(ws + d.off_po);
-  float* part_ml = reinterpret_cast<float*>(ws + d.off_pml);
-  int* err = error_word();
+  int* counters = reinterpret_cast<int*>(ws + d.off_cnt);
   const float scale_log2 = p->scale * 1.4426950408889634f;
   uint16_t* kc = static_cast<uint16_t*>(k_cache);
   uint16_t* vc = static_cast<uint16_t*>(v_cache);
-  uint16_t* kc1 = static_cast<uint16_t*>(kc1_cache);
 
-  decode_append_kernel<<<batch, 128, 0, cs>>>(static_cast<const uint16_t*>(k_new),
-                                               static_cast<const uint16_t*>(v_new), kc, vc, kc1,
-                                               seqlens, p->h_kv, cap, d.cap_c1, err);
-  if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
-  if (d.n_chunks > 0) {
-    dim3 grid(d.n_chunks, p->h_kv, batch);
-    decode_logits_kernel<<<grid, 128, 0, cs>>>(static_cast<const uint16_t*>(q), kc1, seqlens,
-                                                p->h_q, p->h_kv, cap, d.cap_c1, d.zld,
-                                                d.n_chunks, scale_log2, ws_z, ws_ml);
-    if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
-    decode_shared_kernel<<<grid, 256, 0, cs>>>(seqlens, p->h_kv, d.G, cap, d.zld, d.n_chunks,
-                                                d.ld, ws_z, ws_ml, ws_shared);
+  {
+    LogitsArgs a;
+    a.q = static_cast<const uint16_t*>(q);
+    a.k_new = static_cast<const uint16_t*>(k_new);
+    a.v_new = static_cast<const uint16_t*>(v_new);
+    a.k_cache = kc;
+    a.v_cache = vc;
+    a.kc1_cache = static_cast<uint16_t*>(kc1_cache);
+    a.seqlens = seqlens;
+    a.h_q = p->h_q;
+    a.h_kv = p->h_kv;
+    a.cap = cap;
+    a.cap_c1 = d.cap_c1;
+    a.n_chunks = d.n_chunks;
+    a.scale_log2 = scale_log2;
+    a.z = ws_z;
+    a.ml = ws_ml;
+    a.counters = counters;
+    a.err = error_word();
+    dim3 grid(d.n_chunks > 0 ? d.n_chunks : 1, p->h_kv, batch);  // chunk 0 always appends
+    decode_logits_kernel<<<grid, 128, 0, cs>>>(a);
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
   {
-    const int n_keys = (((cap + 63) / 64 + 3) / 4) * 4;
-    const int smem = (n_keys + 256 + 4) * 4;
+    SelectDecArgs a;
+    a.seqlens = seqlens;
+    a.h_kv = p->h_kv;
+    a.G = d.G;
+    a.cap = cap;
+    a.cap_c1 = d.cap_c1;
+    a.n_chunks = d.n_chunks;
+    a.n_init = p->n_init;
+    a.n_local = p->n_local;
+    a.k = p->k;
+    a.z = ws_z;
+    a.ml = ws_ml;
+    a.idx = idx;
+    a.n_keys = (((cap + 63) / 64 + 3) / 4) * 4;
+    const int smem = (a.n_keys + 256 + 4 + 16 + (d.cap_c1 > 0 ? d.cap_c1 : 1)) * 4;
     if (smem > 200 * 1024) return INFV2_ERR_UNSUPPORTED;
     if (!set_smem(decode_select_kernel, smem)) return INFV2_ERR_CUDA;
-    decode_select_kernel<<<batch * p->h_kv, 256, smem, cs>>>(seqlens, p->h_kv, cap, p->n_init,
-                                                              p->n_local, p->k, d.ld, ws_shared,
-                                                              idx, n_keys);
+    decode_select_kernel<<<batch * p->h_kv, 256, smem, cs>>>(a);
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
   {
@@ -371,15 +408,18 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     a.scale_log2 = scale_log2;
     a.decode = 1;
     a.seqlens = seqlens;
+    a.seqlens_out = seqlens;
+    a.cap = cap;
     a.n_split = d.n_split;
-    a.blocks_per_split = kBlocksPerSplit;
+    a.blocks_per_split = d.bps;
     a.split_out = 1;
-    a.part_o = part_o;
-    a.part_ml = part_ml;
+    a.part_o = reinterpret_cast<float*>(ws + d.off_po);
+    a.part_ml = reinterpret_cast<float*>(ws + d.off_pml);
+    a.counters = counters;
+    a.o = static_cast<uint16_t*>(o);
+    a.lse = lse;
     a.wait = wait_ctx();
     if ((st = launch_sparse_attn(tm_k, tm_v, a, cs)) != INFV2_OK) return st;
   }
-  decode_combine_kernel<<<batch, 256, 0, cs>>>(seqlens, p->h_q, cap, d.n_split, part_o, part_ml,
-                                                static_cast<uint16_t*>(o), lse);
-  return launch_status(cudaGetLastError());
+  return INFV2_OK;
 }

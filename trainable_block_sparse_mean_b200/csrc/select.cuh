@@ -145,36 +145,15 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
   __syncwarp();
 }
 
-// Same selection for one row with a whole CTA of 256 threads (used when there
-// are few rows, e.g. one per sequence in decode).  `keys` holds >= bi+1 words,
-// `hist` 256 words and `bcast` 4 words, all in shared memory.
-__device__ __forceinline__ void select_row_cta(const float* __restrict__ row, int nv, int i,
-                                               int n_init, int n_local, int k, uint32_t* keys,
-                                               uint32_t* hist, uint32_t* bcast,
-                                               int* __restrict__ out) {
+// Top-k over block keys already in shared memory (keys[0..bi], forced blocks
+// holding kForcedKey), by a whole CTA: the same exact radix select as above
+// with a CTA-wide histogram.  `hist` 256 words, `bcast` 4 words (shared).
+// Rows with at most k candidates are handled by the caller.
+__device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand, int k,
+                                                uint32_t* hist, uint32_t* bcast,
+                                                int* __restrict__ out) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int bi = i >> 6;
-  const int n_cand = bi + 1;
-  if (n_cand <= k) {
-    for (int b = t; b < k; b += blockDim.x) out[b] = b < n_cand ? b : -1;
-    return;
-  }
-  for (int b = t; b < n_cand; b += blockDim.x) {
-    const int j0 = 4 * b;
-    float m = -INFINITY;
-    if (j0 - 1 >= 0 && j0 - 1 < nv) m = row[j0 - 1];
-    if (j0 + 3 < nv) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(row + j0));
-      m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-    } else {
-      for (int e = 0; e < 3; ++e)
-        if (j0 + e < nv) m = fmaxf(m, row[j0 + e]);
-    }
-    const bool forced = b < n_init || b > bi - n_local;
-    keys[b] = forced ? kForcedKey : float_key(m);
-  }
-  __syncthreads();
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
 #pragma unroll 1
