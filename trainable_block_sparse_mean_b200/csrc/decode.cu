@@ -10,13 +10,15 @@
 //                 K^C1 row (same fp64 mean as prefill compression); every CTA
 //                 computes z = scale*log2(e) * q.K^C1 for its visible kernels
 //                 (stored head-minor) and each head's (max, sum) over the chunk
-//   2. select     (one CTA per (sequence, kv head)): per-head lse from the chunk
+//   2. select     (4 CTAs per (sequence, kv head)): per-head lse from the chunk
 //                 partials, S^shared[j] = sum_h exp2(z_hj - lse_h) for the
-//                 kernels of each block, max pooling and the radix top-k
+//                 kernels of each block, max pooling into block keys; the last
+//                 of the 4 CTAs runs the radix top-k over the row
 //   3. attention  the block-sparse kernel over the selected blocks, the list
-//                 split into pieces of 8 blocks so that several CTAs share a
-//                 sequence; the last piece to finish merges the pieces, writes
-//                 O / lse and, for the last kv head, advances seqlens.
+//                 cut into as many pieces as keep all CTAs in one wave; the
+//                 last piece of a (sequence, kv head) to finish merges the
+//                 pieces, writes O / lse and, for the last kv head, advances
+//                 seqlens.
 #include "attn_sparse.cuh"
 #include "internal.cuh"
 #include "kc1_mean.cuh"
@@ -26,12 +28,12 @@ namespace infv2 {
 namespace {
 
 constexpr int kChunk = 256;         // kernels per logits CTA
-constexpr int kBlocksPerSplit = 8;  // selected blocks per attention CTA (at least)
 constexpr int kMaxPieces = 16;      // pieces the attention kernel's merge accepts
+constexpr int kSelParts = 4;        // CTAs that build one row's block keys
 
 struct DecodePlan {
-  int cap_c1, n_chunks, n_split, bps, G;
-  size_t off_z, off_ml, off_idx, off_po, off_pml, off_cnt, total;
+  int cap_c1, n_chunks, n_keys, G;
+  size_t off_z, off_ml, off_idx, off_po, off_pml, off_keys, off_cnt, total;
 };
 
 DecodePlan plan_decode(const infv2_params* p, int batch, int cap) {
@@ -39,9 +41,7 @@ DecodePlan plan_decode(const infv2_params* p, int batch, int cap) {
   d.G = p->h_q / p->h_kv;
   d.cap_c1 = infv2_num_kernels(p, cap);
   d.n_chunks = (d.cap_c1 + kChunk - 1) / kChunk;
-  d.bps = (p->k + kMaxPieces - 1) / kMaxPieces;
-  if (d.bps < kBlocksPerSplit) d.bps = kBlocksPerSplit;
-  d.n_split = (p->k + d.bps - 1) / d.bps;
+  d.n_keys = (((cap + 63) / 64 + 3) / 4) * 4;
   size_t off = 0;
   d.off_z = off;  // [batch][h_kv][cap_c1][16] logits, heads padded to 16
   off += round256((size_t)batch * p->h_kv * (d.cap_c1 > 0 ? d.cap_c1 : 1) * 16 * 4);
@@ -49,12 +49,15 @@ DecodePlan plan_decode(const infv2_params* p, int batch, int cap) {
   off += round256((size_t)batch * p->h_kv * (d.n_chunks > 0 ? d.n_chunks : 1) * 16 * 2 * 4);
   d.off_idx = off;
   off += round256((size_t)batch * p->h_kv * p->k * 4);
-  d.off_po = off;
-  off += round256((size_t)batch * p->h_q * d.n_split * 128 * 4);
+  d.off_po = off;  // attention pieces (at most kMaxPieces per row)
+  off += round256((size_t)batch * p->h_q * kMaxPieces * 128 * 4);
   d.off_pml = off;
-  off += round256((size_t)batch * p->h_q * d.n_split * 2 * 4);
-  d.off_cnt = off;  // split counters [batch][h_kv], sequence counters [batch]
-  off += round256((size_t)batch * (p->h_kv + 1) * 4);
+  off += round256((size_t)batch * p->h_q * kMaxPieces * 2 * 4);
+  d.off_keys = off;  // block keys of each row, built by kSelParts CTAs
+  off += round256((size_t)batch * p->h_kv * d.n_keys * 4);
+  d.off_cnt = off;  // attention piece counters [batch][h_kv], row counters [batch],
+                    // selection part counters [batch][h_kv]
+  off += round256((size_t)batch * (2 * p->h_kv + 1) * 4);
   d.total = off;
   return d;
 }
@@ -106,8 +109,10 @@ __global__ void __launch_bounds__(128) decode_logits_kernel(LogitsArgs a) {
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
     }
     if (t == 32) {
-      a.counters[sg] = 0;
-      if (g == 0) a.counters[(size_t)gridDim.z * a.h_kv + s] = 0;
+      const size_t B = gridDim.z;
+      a.counters[sg] = 0;                                   // attention pieces
+      if (g == 0) a.counters[B * a.h_kv + s] = 0;           // attention rows
+      a.counters[B * (a.h_kv + 1) + sg] = 0;                // selection parts
     }
   }
   const int nv = visible_kernels(L, 32, 16);  // includes a kernel completed by token L
@@ -145,18 +150,28 @@ __global__ void __launch_bounds__(128) decode_logits_kernel(LogitsArgs a) {
   float* zbase = a.z + sg * a.cap_c1 * 16;
   float mx0 = -INFINITY, mx1 = -INFINITY;
   float zv[8][4];
+  // the next n-tile's K^C1 rows are loaded while the current one is used
+  // (L2-only loads: this kernel may have written a row)
+  uint4 kn[4];
+  {
+    const int jr = j_chunk + warp * 64 + gid;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      kn[c] = jr < nv ? __ldcg(reinterpret_cast<const uint4*>(kbase + (size_t)jr * 128 + 32 * c))
+                      : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
     const int jn = j_chunk + warp * 64 + nt * 8;  // first kernel of this n-tile
-    const int jr = jn + gid;                      // kernel row this lane loads
     uint4 kv[4];
-    if (jr < nv) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)  // L2-only loads: this kernel may have written the row
-        kv[c] = __ldcg(reinterpret_cast<const uint4*>(kbase + (size_t)jr * 128 + 32 * c));
-    } else {
+    for (int c = 0; c < 4; ++c) kv[c] = kn[c];
+    if (nt + 1 < 8) {
+      const int jr = jn + 8 + gid;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) kv[c] = make_uint4(0u, 0u, 0u, 0u);
+      for (int c = 0; c < 4; ++c)
+        kn[c] = jr < nv ? __ldcg(reinterpret_cast<const uint4*>(kbase + (size_t)jr * 128 + 32 * c))
+                        : make_uint4(0u, 0u, 0u, 0u);
     }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -217,32 +232,39 @@ struct SelectDecArgs {
   int n_init, n_local, k;
   const float* z;
   const float* ml;
-  int* idx;  // [batch, h_kv, k]
+  uint32_t* keys_g;  // [batch * h_kv][n_keys]
+  int* part_cnt;     // [batch * h_kv]
+  int* idx;          // [batch, h_kv, k]
   int n_keys;
 };
 
-// 2. per-head lse, S^shared per block window, max pooling and top-k for one
-// (sequence, kv head), by a CTA of 256 threads.
+// 2. selection for one (sequence, kv head), spread over kSelParts CTAs of 256
+// threads: each part computes the per-head lse, S^shared[j] = sum_h
+// exp2(z_hj - lse_h) for the kernels of its blocks and their max-pooled keys;
+// the last part to finish runs the radix top-k over the whole row.
 __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
   extern __shared__ __align__(16) uint32_t sm_sel[];
-  uint32_t* keys = sm_sel;
-  uint32_t* hist = keys + a.n_keys;
-  uint32_t* bcast = hist + 256;
+  __shared__ int s_last;
+  uint32_t* keys = sm_sel;                            // [n_keys]
+  uint32_t* hist = keys + a.n_keys;                   // [256]
+  uint32_t* bcast = hist + 256;                       // [4]
   float* lse2 = reinterpret_cast<float*>(bcast + 4);  // [16]
-  float* shared_s = lse2 + 16;                        // [cap_c1] S^shared of the row
-  const int sgi = blockIdx.x;
+  float* shared_s = lse2 + 16;                        // S^shared of this part's kernels
+  const int part = blockIdx.x, sgi = blockIdx.y;
   const int s = sgi / a.h_kv;
   const int t = threadIdx.x;
   const int L = a.seqlens[s];
   int* out = a.idx + (size_t)sgi * a.k;
   if (L < 0 || L >= a.cap) {
-    for (int x = t; x < a.k; x += blockDim.x) out[x] = -1;
+    if (part == 0)
+      for (int x = t; x < a.k; x += blockDim.x) out[x] = -1;
     return;
   }
   const int bi = L >> 6;
   const int n_cand = bi + 1;
   if (n_cand <= a.k) {  // every visible block
-    for (int b = t; b < a.k; b += blockDim.x) out[b] = b < n_cand ? b : -1;
+    if (part == 0)
+      for (int b = t; b < a.k; b += blockDim.x) out[b] = b < n_cand ? b : -1;
     return;
   }
   const int nv = visible_kernels(L, 32, 16);
@@ -267,16 +289,20 @@ __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
   float lse_r[16];
 #pragma unroll
   for (int h = 0; h < 16; ++h) lse_r[h] = lse2[h];
-  // S^shared of every visible kernel into shared memory; each thread keeps
-  // the logit loads of four kernels in flight
+  // this part's blocks and the kernels intersecting them
+  const int per = (n_cand + kSelParts - 1) / kSelParts;
+  const int b_lo = part * per;
+  const int b_hi = min(n_cand, b_lo + per);
+  const int j_lo = max(0, 4 * b_lo - 1);
+  const int j_hi = min(nv, 4 * b_hi + 3);  // exclusive
   const float* zrow = a.z + (size_t)sgi * a.cap_c1 * 16;
   const int G = a.G;
-  for (int j0 = t; j0 < nv; j0 += 4 * blockDim.x) {
+  for (int j0 = j_lo + t; j0 < j_hi; j0 += 4 * blockDim.x) {
     float4 v[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u * blockDim.x;
-      const float4* zr = reinterpret_cast<const float4*>(zrow + (size_t)(j < nv ? j : 0) * 16);
+      const float4* zr = reinterpret_cast<const float4*>(zrow + (size_t)(j < j_hi ? j : j_lo) * 16);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4)
         v[u][q4] = 4 * q4 < G ? __ldg(zr + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -292,19 +318,27 @@ __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
         for (int e = 0; e < 4; ++e)
           if (4 * q4 + e < G) sh += fast_exp2(vv[e] - lse_r[4 * q4 + e]);
       }
-      if (j < nv) shared_s[j] = sh;
+      if (j < j_hi) shared_s[j - j_lo] = sh;
     }
   }
   __syncthreads();
-  // max pooling over the kernels intersecting each block (4b-1 .. 4b+3)
-  for (int b = t; b < n_cand; b += blockDim.x) {
+  uint32_t* kg = a.keys_g + (size_t)sgi * a.n_keys;
+  for (int b = b_lo + t; b < b_hi; b += blockDim.x) {
     const bool forced = b < a.n_init || b > bi - a.n_local;
     float m = -INFINITY;
 #pragma unroll
     for (int j = 4 * b - 1; j <= 4 * b + 3; ++j)
-      if (j >= 0 && j < nv) m = fmaxf(m, shared_s[j]);
-    keys[b] = forced ? kForcedKey : float_key(m);
+      if (j >= j_lo && j < j_hi) m = fmaxf(m, shared_s[j - j_lo]);
+    kg[b] = forced ? kForcedKey : float_key(m);
   }
+  __threadfence();  // this part's keys are visible before it is counted
+  __syncthreads();
+  if (t == 0) s_last = atomicAdd(&a.part_cnt[sgi], 1) == kSelParts - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int b = t; b < n_cand; b += blockDim.x) keys[b] = __ldcg(kg + b);
+  if (t == 0) a.part_cnt[sgi] = 0;
   __syncthreads();
   select_topk_cta(keys, n_cand, a.k, hist, bcast, out);
 }
@@ -382,12 +416,15 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     a.k = p->k;
     a.z = ws_z;
     a.ml = ws_ml;
+    a.keys_g = reinterpret_cast<uint32_t*>(ws + d.off_keys);
+    a.part_cnt = counters + (size_t)batch * (p->h_kv + 1);
     a.idx = idx;
-    a.n_keys = (((cap + 63) / 64 + 3) / 4) * 4;
-    const int smem = (a.n_keys + 256 + 4 + 16 + (d.cap_c1 > 0 ? d.cap_c1 : 1)) * 4;
+    a.n_keys = d.n_keys;
+    const int part_kernels = 4 * ((d.n_keys + kSelParts - 1) / kSelParts) + 8;
+    const int smem = (a.n_keys + 256 + 4 + 16 + part_kernels) * 4;
     if (smem > 200 * 1024) return INFV2_ERR_UNSUPPORTED;
     if (!set_smem(decode_select_kernel, smem)) return INFV2_ERR_CUDA;
-    decode_select_kernel<<<batch * p->h_kv, 256, smem, cs>>>(a);
+    decode_select_kernel<<<dim3(kSelParts, batch * p->h_kv), 256, smem, cs>>>(a);
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
   {
@@ -410,8 +447,14 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     a.seqlens = seqlens;
     a.seqlens_out = seqlens;
     a.cap = cap;
-    a.n_split = d.n_split;
-    a.blocks_per_split = d.bps;
+    // as many pieces per row as keep the whole step in one wave of CTAs
+    int pieces = (2 * sm_count()) / (batch * p->h_kv);
+    if (pieces > kMaxPieces) pieces = kMaxPieces;
+    if (pieces > p->k) pieces = p->k;
+    if (pieces < 1) pieces = 1;
+    const int bps = (p->k + pieces - 1) / pieces;
+    a.n_split = (p->k + bps - 1) / bps;
+    a.blocks_per_split = bps;
     a.split_out = 1;
     a.part_o = reinterpret_cast<float*>(ws + d.off_po);
     a.part_ml = reinterpret_cast<float*>(ws + d.off_pml);
