@@ -249,6 +249,7 @@ def run_ours(args, rank, world, local_rank, dist):
                 "launches_per_step": launches_per_step}
     # ---- per-stage breakdown on the same stream (CUDA events between launches)
     stage = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows)
+    fused = _fused_pool_timing(args, infv2, torch, p, shape, q, k, ws, stream, chunk_rows, stage)
     # ---- end to end through host buffers
     e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_ranks)
     # ---- decode
@@ -302,6 +303,7 @@ def run_ours(args, rank, world, local_rank, dist):
                                        "attention": round(work["attn"] / 1e12, 3)},
         "selection_share": round(sel_ms / stage["ms_per_step"], 4),
         "stages": stage["per_kernel"],
+        "fused_pool": fused,
         "roofline": roof,
         "e2e": e2e,
         "decode": dec,
@@ -385,6 +387,48 @@ def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, 
     for nm in names:
         per[nm] = {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in per[nm].items()}
     return dict(per_kernel=per, ms_per_step=e0.elapsed_time(e1) / steps)
+
+
+def _fused_pool_timing(args, infv2, torch, p, shape, q, k, ws, stream, chunk_rows, stage):
+    """The alternative stage 2-4 path with max pooling fused into the score
+    kernel (block scores S^cmp out, top-k-only selection), timed over the same
+    row chunks as the unfused stages; reported beside them, not in the step."""
+    n = shape.n
+    nc = infv2.num_kernels(p, n)
+    ldc = infv2.cmp_ld(n)
+    kc1 = ws[: nc * p.h_kv * 128 * 2].view(torch.bfloat16).view(nc, p.h_kv, 128)
+    off = ((nc * p.h_kv * 256) + 255) // 256 * 256
+    s_cmp = ws[off: off + p.h_kv * chunk_rows * ldc * 4].view(torch.float32)
+    idx = torch.empty((p.h_kv, n, p.k), dtype=torch.int32, device=q.device)
+    infv2.infv2_compress_k(p, k, kc1)
+
+    def one():
+        evs = []
+        for q0 in range(0, n, chunk_rows):
+            ql = min(chunk_rows, n - q0)
+            buf = s_cmp[: p.h_kv * ql * ldc].view(p.h_kv, ql, ldc)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            c = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            infv2.infv2_block_scores_pooled(p, q, kc1, n, q0, ql, buf, ldc)
+            b.record(stream)
+            infv2.infv2_select_topk_pooled(p, buf, ldc, n, q0, ql, idx)
+            c.record(stream)
+            evs.append((a, b, c))
+        return evs
+
+    one()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    runs = [one() for _ in range(steps)]
+    torch.cuda.synchronize()
+    sc = sum(a.elapsed_time(b) for r in runs for a, b, _ in r) / steps
+    se = sum(b.elapsed_time(c) for r in runs for _, b, c in r) / steps
+    unfused = stage["per_kernel"]["score_kernel"]["ms_per_step"] + stage["per_kernel"]["select_kernel"]["ms_per_step"]
+    return {"score_kernel_pooled_ms_per_step": round(sc, 4), "select_pooled_kernel_ms_per_step": round(se, 4),
+            "total_ms_per_step": round(sc + se, 4), "unfused_total_ms_per_step": round(unfused, 4),
+            "chunk_rows": chunk_rows, "used_in_step": False}
 
 
 def _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks):

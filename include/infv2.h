@@ -135,6 +135,26 @@ int infv2_block_scores(const infv2_params* p, const void* q, const void* kc1, in
 int infv2_select_topk(const infv2_params* p, const float* s_shared, int ld, int n, int q_begin,
                       int q_len, int* idx, infv2_stream_t stream);
 
+/* Stages 2-3 fused (paper notes, limitations: folding max pooling and top-k
+ * into the kernel is left as future work there).  Same computation as
+ * infv2_block_scores followed by the max pooling of infv2_select_topk, done
+ * in the score kernel's epilogue, so only the block scores reach memory:
+ *   s_cmp   fp32 [h_kv, q_len, ld_cmp] (output): row (g, i - q_begin) holds
+ *           S^cmp[b] for b < i/B (the blocks before the query's own block,
+ *           which is always a local block); entries from i/B on are not
+ *           written.  ld_cmp >= ceil(n / B) and a multiple of 4.
+ * Other arguments as infv2_block_scores (no score_lse output). */
+int infv2_block_scores_pooled(const infv2_params* p, const void* q, const void* kc1, int n,
+                              int q_begin, int q_len, float* s_cmp, int ld_cmp,
+                              infv2_stream_t stream);
+
+/* Stage 4 alone: the top-k selection of infv2_select_topk from the block
+ * scores written by infv2_block_scores_pooled (same rule, same output).
+ *   s_cmp  fp32 [h_kv, q_len, ld_cmp], 16-byte aligned, ld_cmp a multiple
+ *          of 4;  idx int32 [h_kv, n, k] (output). */
+int infv2_select_topk_pooled(const infv2_params* p, const float* s_cmp, int ld_cmp, int n,
+                             int q_begin, int q_len, int* idx, infv2_stream_t stream);
+
 /* Stage 5, block-sparse attention (arXiv summary, Appendix A): for every
  * query i and head h of group g, softmax attention over the tokens t <= i of
  * the blocks listed in idx[g, i, :] (entries < 0 ignored).

@@ -98,6 +98,14 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_block_scores(P, None, None, 100, 50, 60, None, 128, None, None) == infv2.ERR_INVALID_ARG
     assert L.infv2_select_topk(P, None, 128, 100, 0, 0, None, None) == infv2.OK
     assert L.infv2_select_topk(P, None, 6, 100, 0, 10, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_block_scores_pooled(P, None, None, 100, 50, 60, None, 4, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_block_scores_pooled(P, None, None, 100, 0, 0, None, 4, None) == infv2.OK
+    # ld_cmp below ceil(n/B) or not a multiple of 4 is rejected before any pointer is used
+    assert L.infv2_block_scores_pooled(P, 16, 16, 1000, 0, 10, 16, 12, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_block_scores_pooled(P, 16, 16, 1000, 0, 10, 16, 18, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_select_topk_pooled(P, None, 4, 100, 0, 0, None, None) == infv2.OK
+    assert L.infv2_select_topk_pooled(P, 16, 2, 100, 0, 10, 16, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_select_topk_pooled(P, 8, 4, 100, 0, 10, 16, None) == infv2.ERR_INVALID_ARG  # misaligned
     assert L.infv2_sparse_attn(P, None, None, None, None, 10, None, None, None) == infv2.ERR_INVALID_ARG
     assert L.infv2_dense_attn(P, None, None, None, 0, None, None, None) == infv2.OK
     assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,

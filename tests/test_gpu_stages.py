@@ -104,6 +104,79 @@ def test_block_scores_match_oracle(n, h_q, h_kv, q_begin, q_len):
             assert np.allclose(lg, lw, rtol=0, atol=2e-5), (i, lg - lw)
 
 
+@pytest.mark.parametrize("n,h_q,h_kv,q_begin,q_len", [
+    (2048, 4, 1, 0, 2048),        # G=4, one kernel tile: carries between warp quarters
+    (3000, 32, 2, 0, 3000),       # G=16, ragged tail
+    (3000, 32, 2, 1000, 1333),    # a chunk in the middle of the sequence
+    (700, 8, 1, 0, 700),          # G=8
+    (600, 2, 2, 0, 600),          # G=1
+    (900, 4, 2, 0, 900),          # G=2
+    (17000, 32, 2, 16000, 1000),  # 9 kernel tiles: windows across tile boundaries
+])
+def test_pooled_block_scores_match_oracle(n, h_q, h_kv, q_begin, q_len):
+    """Scores with max pooling fused into the score kernel: S^cmp[b] for b < i/B."""
+    sh, d = _problem(n, h_q, h_kv, seed=n + 3 * h_q)
+    p = infv2.params_of(sh)
+    op = oracle.params(sh)
+    kc1 = infv2.infv2_compress_k(p, to_dev(d["k"]))
+    ldc = infv2.cmp_ld(n)
+    sentinel = 7.25
+    s = torch.full((h_kv, q_len, ldc), sentinel, device="cuda")
+    infv2.infv2_block_scores_pooled(p, to_dev(d["q"]), kc1, n, q_begin, q_len, s, ldc)
+    # the unfused scores of the same kernel, pooled on the host in fp32
+    ld = infv2.shared_ld(n)
+    full = infv2.infv2_block_scores(p, to_dev(d["q"]), kc1, n, q_begin, q_len, ld=ld)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    s = s.cpu().numpy()
+    full = full.cpu().numpy()
+    rows = _sample_rows(n, 40, seed=n + 1)
+    rows = rows[(rows >= q_begin) & (rows < q_begin + q_len)]
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows, want_cmp=True)
+    for r, i in enumerate(rows):
+        nb = int(i) // 64
+        nv = oracle.visible_kernels(op, i)
+        for g in range(h_kv):
+            got = s[g, i - q_begin, :nb]
+            want = ref["cmp"][r, g, :nb]
+            err = np.abs(got - want) / np.maximum(np.abs(want), 1e-30)
+            assert err.max(initial=0) <= SCORE_REL, (i, g, err.max(), int(err.argmax()))
+            assert np.all(s[g, i - q_begin, nb:] == sentinel)   # own block onwards untouched
+            row = full[g, i - q_begin, :nv]
+            pooled = np.array([row[max(4 * b - 1, 0):min(4 * b + 4, nv)].max() for b in range(nb)],
+                              np.float32)
+            assert np.array_equal(got, pooled), (i, g)
+
+
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64)])
+def test_select_pooled_exact_on_oracle_scores(n, h_q, h_kv, k):
+    """Top-k from S^cmp, decided on the same fp32 values as the oracle."""
+    sh, d = _problem(n, h_q, h_kv, k=k, seed=4)
+    op = oracle.params(sh)
+    p = infv2.params_of(sh)
+    rows = _sample_rows(n, 200, seed=2)
+    ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows, want_cmp=True)
+    c32 = ref["cmp"].astype(np.float32)               # [rows, h_kv, n_blk]
+    ties = np.round(c32 * 32) / 32
+    n_blk = c32.shape[2]
+    ldc = infv2.cmp_ld(n)
+    for vals in (c32, ties):
+        buf = np.full((h_kv, len(rows), ldc), np.nan, np.float32)
+        for r, i in enumerate(rows):   # only b < i/B is defined; the rest stays NaN
+            buf[:, r, :int(i) // 64] = vals[r, :, :int(i) // 64]
+        dev = torch.from_numpy(buf).cuda()
+        idx = torch.full((h_kv, n, k), -2, dtype=torch.int32, device="cuda")
+        for r, i in enumerate(rows):
+            infv2.infv2_select_topk_pooled(p, dev[:, r:r + 1, :].contiguous(), ldc, n, int(i), 1, idx)
+        torch.cuda.synchronize()
+        idx = idx.cpu().numpy()
+        for r, i in enumerate(rows):
+            for g in range(h_kv):
+                want = oracle.select_row(op, vals[r, g, :int(i) // 64 + 1].astype(np.float64), int(i))
+                assert np.array_equal(idx[g, i, :], want), (i, g)
+        assert n_blk == (n + 63) // 64
+
+
 # ---------------------------------------------------------------- stages 3-4
 
 @pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64)])
@@ -166,6 +239,35 @@ def test_sparse_attn_on_oracle_indices(n, h_q, h_kv, k):
             first = og
         else:
             assert np.array_equal(og, first), "sparse_attn is not deterministic"
+
+
+def test_sparse_attn_lists_with_holes():
+    """Entries < 0 anywhere in a list are ignored; neighbouring tokens with
+    overlapping and disjoint lists share the fetched blocks."""
+    n, h_q, h_kv, k = 1999, 32, 2, 16
+    sh, d = _problem(n, h_q, h_kv, k=k, seed=23)
+    op = oracle.params(sh)
+    p = infv2.params_of(sh)
+    rng = np.random.default_rng(4)
+    idx = np.full((h_kv, n, k), -1, np.int32)
+    for g in range(h_kv):
+        for i in range(n):
+            nb = i // 64 + 1
+            cnt = min(nb, int(rng.integers(1, k + 1)))
+            chosen = np.sort(rng.choice(nb, size=cnt, replace=False))
+            slots = np.sort(rng.choice(k, size=cnt, replace=False))   # -1 holes between them
+            idx[g, i, slots] = chosen
+    rows = _sample_rows(n, 120, seed=6)
+    want_o, want_lse = oracle.attend_rows(op, d["q"], d["k"], d["v"], rows,
+                                          idx[:, rows, :].transpose(1, 0, 2).copy())
+    lse = torch.empty((h_q, n), device="cuda")
+    o = infv2.infv2_sparse_attn(p, to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]),
+                                torch.from_numpy(idx).cuda(), lse=lse)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    og = synth.bf16_to_f32(to_host_bits(o))[rows]
+    parity.assert_outputs_close(og, want_o, "sparse_attn holes")
+    assert np.allclose(lse.cpu().numpy()[:, rows].T, want_lse, rtol=0, atol=2e-3)
 
 
 @pytest.mark.parametrize("n,h_q,h_kv", [(1024, 32, 2), (777, 4, 1), (64, 16, 2), (1, 2, 1), (130, 8, 2)])

@@ -13,6 +13,19 @@ int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t
 int launch_select(const infv2_params* p, const float* s_shared, int ld, int n, int q_begin,
                   int q_len, int* idx, long long idx_hstride, cudaStream_t st);
 
+// Fused form: block scores S^cmp [h_kv, q_len, ld_cmp] straight from the score
+// kernel (max pooling in its epilogue), then a top-k-only selection.
+int launch_block_scores_pooled(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
+                               int n, int q_begin, int q_len, float* s_cmp, int ld_cmp,
+                               cudaStream_t st);
+
+int launch_select_pooled(const infv2_params* p, const float* s_cmp, int ld_cmp, int n,
+                         int q_begin, int q_len, int* idx, long long idx_hstride,
+                         cudaStream_t st);
+
+// Row pitch (floats) of S^cmp: blocks of an n-token sequence rounded to 32.
+inline int cmp_ld(int n) { return (((n + 63) / 64) + 31) / 32 * 32; }
+
 // Row pitch (floats) of S^shared for an n-token sequence: at least the kernel
 // count and four kernels per block, rounded to 32 floats (128 bytes).
 inline int shared_ld(int n) {

@@ -43,7 +43,9 @@ struct ScoreArgs {
   int q_begin, q_len, n_tiles;
   float scale_log2;     // scale * log2(e)
   int ld;
-  float* s_shared;      // [h_kv, q_len, ld]
+  float* s_shared;      // [h_kv, q_len, ld]      (unpooled form)
+  float* s_cmp;         // [h_kv, q_len, ld_cmp]  (pooled form: block scores)
+  int ld_cmp;
   float* score_lse;     // [h_q, q_len] or null
   WaitCtx wait;
 };
@@ -53,18 +55,30 @@ struct ScoreSmem {
   uint32_t q_full, kv_full, kv_empty, acc_full, acc_empty, lse_ready;  // barriers (8 B each)
 };
 
-template <int G>
+// POOL: instead of S^shared, write the block scores S^cmp[b] = max of S^shared
+// over the kernels 4b-1 .. 4b+3 (those intersecting block b).  In pass 2 a
+// TMEM lane owns one kernel, so kernels 4b .. 4b+3 are four aligned lanes of a
+// warp (shuffle max) and kernel 4b-1 is the previous lane; the first lane of a
+// warp takes it from the previous warp quarter (or the previous tile's last
+// quarter) through shared memory: the four warps of a column group publish
+// their last lane per tile and meet on a bounded mbarrier.  Tile t uses
+// exchange slot t%3, read at tiles t and t+1; it is rewritten at tile t+3 only
+// after the writer has passed the barrier of tile t+2, which every warp
+// reaches after its reads at tile t+1.
+template <int G, bool POOL>
 __global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  ScoreArgs a) {
   constexpr int TQ = 128 / G;
+  constexpr int TPG = kCols / G > 0 ? kCols / G : 1;  // tokens per column group
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   float* s_lse2 = reinterpret_cast<float*>(base + kTileBytes * (1 + kStages));
   float* s_part = s_lse2 + 128;  // [column group][128 rows][max, sum]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_part + kColGroups * 128 * 2);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4);
+  float* s_xch = s_part + kColGroups * 128 * 2;        // [3][kColGroups][4 quarters][TPG]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_xch + 3 * kColGroups * 4 * TPG + 2);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4 + kColGroups);
   ScoreSmem S;
   S.q = smem_u32(base);
   S.k = S.q + kTileBytes;
@@ -74,6 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   S.acc_full = S.kv_empty + 8 * kStages;
   S.acc_empty = S.acc_full + 16;
   S.lse_ready = S.acc_empty + 16;
+  const uint32_t cg_bar0 = S.lse_ready + 8;  // POOL: one barrier per column group
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -104,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(S.acc_empty + 8 * b, kEpiWarps);
     }
     mbar_init(S.lse_ready, kEpiWarps);
+    if (POOL)
+      for (int x = 0; x < kColGroups; ++x) mbar_init(cg_bar0 + 8 * x, 4);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -181,6 +198,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = a.scale_log2;
     float vmax = -INFINITY, l = 0.f;
     float* out_g = a.s_shared + (size_t)g * a.q_len * a.ld;
+    // POOL: per token of this column group, the S^cmp row and the number of
+    // blocks it holds (i/B; 0 for rows past the tile's end)
+    float* cmp_row[TPG];
+    int cmp_lim[TPG];
+    int slot = 0, slot_prev = 2;  // POOL: exchange slots of this tile and the previous one
+    if constexpr (POOL) {
+#pragma unroll
+      for (int t = 0; t < TPG; ++t) {
+        const int i = i0 + cg * TPG + t;
+        const bool in = i <= i_last;
+        cmp_row[t] = a.s_cmp + ((size_t)g * a.q_len + (in ? i - a.q_begin : 0)) * a.ld_cmp;
+        cmp_lim[t] = in ? (i >> 6) : 0;
+      }
+    }
     for (int it = 0; it < total_it; ++it) {
       const int b = it & 1;
       if (!mbar_wait(S.acc_full + 8 * b, (it >> 1) & 1, a.wait)) break;
@@ -247,10 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // pass 2: kernel j = (it - n_kt)*128 + r; this group's columns = tokens
-        const int j = (it - n_kt) * 128 + r;
-        constexpr int TPG = kCols / G > 0 ? kCols / G : 1;  // tokens per column group
+        const int jt = it - n_kt;
+        const int j = jt * 128 + r;
         static_assert(G <= kCols, "a token's heads must fit in one column group");
         const float4* lse4 = reinterpret_cast<const float4*>(s_lse2 + cg * kCols);
+        float pv[TPG];  // POOL: this kernel's S^shared per token (-inf if not visible)
 #pragma unroll
         for (int t = 0; t < TPG; ++t) {
           const int tq = cg * TPG + t;
@@ -271,8 +303,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               ps[hh] += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
           }
           const float ssum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-          if (i <= i_last && j < visible_kernels(i, 32, 16))
-            out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
+          const bool vis = i <= i_last && j < visible_kernels(i, 32, 16);
+          if constexpr (POOL) {
+            pv[t] = vis ? ssum : -INFINITY;
+          } else {
+            if (vis) out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
+          }
+        }
+        if constexpr (POOL) {
+          float* xch = s_xch + ((slot * kColGroups + cg) * 4) * TPG;
+          if (lane == 31)
+#pragma unroll
+            for (int t = 0; t < TPG; ++t) xch[quarter * TPG + t] = pv[t];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(cg_bar0 + 8 * cg);
+          if (!mbar_wait(cg_bar0 + 8 * cg, (uint32_t)(jt & 1), a.wait)) break;
+          // kernel 4b-1 for lane 0: the previous quarter's last lane, or the
+          // previous tile's last quarter
+          const float* prv = quarter > 0 ? xch + (quarter - 1) * TPG
+                                         : s_xch + ((slot_prev * kColGroups + cg) * 4 + 3) * TPG;
+          slot_prev = slot;
+          slot = slot == 2 ? 0 : slot + 1;
+          const int b = j >> 2;
+#pragma unroll
+          for (int t = 0; t < TPG; ++t) {
+            float prev = __shfl_up_sync(0xFFFFFFFFu, pv[t], 1);
+            if (lane == 0) prev = (quarter > 0 || jt > 0) ? prv[t] : -INFINITY;
+            float m4 = fmaxf(pv[t], __shfl_xor_sync(0xFFFFFFFFu, pv[t], 1));
+            m4 = fmaxf(m4, __shfl_xor_sync(0xFFFFFFFFu, m4, 2));  // kernels 4b .. 4b+3
+            if ((lane & 3) == 0 && b < cmp_lim[t]) cmp_row[t][b] = fmaxf(m4, prev);
+          }
         }
       }
     }
@@ -285,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int G>
+template <int G, bool POOL>
 int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h_kv, int q_begin,
-                   int q_len, float scale, float* s_shared, int ld, float* score_lse,
+                   int q_len, float scale, float* s_out, int ld, float* score_lse,
                    cudaStream_t st) {
   constexpr int TQ = 128 / G;
   const int nc = n >= 32 ? (n - 32) / 16 + 1 : 0;
@@ -297,21 +357,40 @@ int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h
   // K^C1 map; an empty K^C1 (nc == 0) still needs a valid map, one row is enough
   if (!make_tmap_3d(&tm_k, kc1, 128, h_kv, nc > 0 ? nc : 1, 256, (uint64_t)h_kv * 256, 64, 1, 128))
     return INFV2_ERR_CUDA;
+  constexpr int TPG = kCols / G > 0 ? kCols / G : 1;
   const int smem = kTileBytes * (1 + kStages) + 128 * 4 + kColGroups * 128 * 2 * 4 +
-                   8 * (2 + 2 * kStages + 4) + 16 + 1024;
-  if (!set_smem(score_kernel<G>, smem)) return INFV2_ERR_CUDA;
+                   (3 * kColGroups * 4 * TPG + 2) * 4 +
+                   8 * (2 + 2 * kStages + 4 + kColGroups) + 16 + 1024;
+  if (!set_smem(score_kernel<G, POOL>, smem)) return INFV2_ERR_CUDA;
   ScoreArgs a;
   a.q_begin = q_begin;
   a.q_len = q_len;
   a.n_tiles = (q_len + TQ - 1) / TQ;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.ld = ld;
-  a.s_shared = s_shared;
+  a.s_shared = POOL ? nullptr : s_out;
+  a.s_cmp = POOL ? s_out : nullptr;
+  a.ld_cmp = ld;
   a.score_lse = score_lse;
   a.wait = wait_ctx();
   dim3 grid(a.n_tiles, h_kv);
-  score_kernel<G><<<grid, kThreads, smem, st>>>(tm_q, tm_k, a);
+  score_kernel<G, POOL><<<grid, kThreads, smem, st>>>(tm_q, tm_k, a);
   return launch_status(cudaGetLastError());
+}
+
+template <bool POOL>
+int launch_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
+                  int q_begin, int q_len, float* out, int ld, float* score_lse, cudaStream_t st) {
+  if (q_len <= 0) return INFV2_OK;
+  const int G = p->h_q / p->h_kv;
+  switch (G) {
+    case 1: return launch_score_g<1, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+    case 2: return launch_score_g<2, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+    case 4: return launch_score_g<4, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+    case 8: return launch_score_g<8, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+    case 16: return launch_score_g<16, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+    default: return INFV2_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace
@@ -319,16 +398,13 @@ int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h
 int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
                         int q_begin, int q_len, float* s_shared, int ld, float* score_lse,
                         cudaStream_t st) {
-  if (q_len <= 0) return INFV2_OK;
-  const int G = p->h_q / p->h_kv;
-  switch (G) {
-    case 1: return launch_score_g<1>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
-    case 2: return launch_score_g<2>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
-    case 4: return launch_score_g<4>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
-    case 8: return launch_score_g<8>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
-    case 16: return launch_score_g<16>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, s_shared, ld, score_lse, st);
-    default: return INFV2_ERR_UNSUPPORTED;
-  }
+  return launch_scores<false>(p, q, kc1, n, q_begin, q_len, s_shared, ld, score_lse, st);
+}
+
+int launch_block_scores_pooled(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
+                               int n, int q_begin, int q_len, float* s_cmp, int ld_cmp,
+                               cudaStream_t st) {
+  return launch_scores<true>(p, q, kc1, n, q_begin, q_len, s_cmp, ld_cmp, nullptr, st);
 }
 
 }  // namespace infv2
@@ -351,4 +427,21 @@ extern "C" int infv2_block_scores(const infv2_params* p, const void* q, const vo
   return launch_block_scores(p, static_cast<const uint16_t*>(q),
                              static_cast<const uint16_t*>(kc1_map), n, q_begin, q_len, s_shared,
                              ld, score_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int infv2_block_scores_pooled(const infv2_params* p, const void* q, const void* kc1,
+                                         int n, int q_begin, int q_len, float* s_cmp, int ld_cmp,
+                                         infv2_stream_t stream) {
+  int st = infv2_check_params(p);
+  if (st != INFV2_OK) return st;
+  if (n < 0 || q_begin < 0 || q_len < 0 || q_begin + q_len > n) return INFV2_ERR_INVALID_ARG;
+  if (q_len == 0) return INFV2_OK;
+  if (!q || !s_cmp) return INFV2_ERR_INVALID_ARG;
+  const int nc = infv2_num_kernels(p, n);
+  if (nc > 0 && !kc1) return INFV2_ERR_INVALID_ARG;
+  if (ld_cmp < (n + p->B - 1) / p->B || ld_cmp % 4 != 0) return INFV2_ERR_INVALID_ARG;
+  if (nc == 0) return INFV2_OK;  // no block has a visible kernel
+  return launch_block_scores_pooled(p, static_cast<const uint16_t*>(q),
+                                    static_cast<const uint16_t*>(kc1), n, q_begin, q_len, s_cmp,
+                                    ld_cmp, reinterpret_cast<cudaStream_t>(stream));
 }

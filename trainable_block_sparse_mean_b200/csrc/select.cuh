@@ -25,57 +25,11 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 
 constexpr uint32_t kForcedKey = 0xFFFFFFFFu;  // above every finite score and +inf
 
-// Select for one row.  `row` holds S^shared[j] for j < nv (entries at
-// j >= nv may be garbage and are never used; reads stay below 4*(bi+1)).
-// `keys` is per-warp shared scratch of >= bi+1 words, `hist` 256 words.
-// Writes k indices (ascending, -1 padded) to `out`.
-__device__ __forceinline__ void select_row_warp(const float* __restrict__ row, int nv, int i,
-                                                int n_init, int n_local, int k, uint32_t* keys,
-                                                uint32_t* hist, int* __restrict__ out) {
+// Exact top-k of keys[0 .. n_cand) (per-warp shared memory) by one warp:
+// ascending block indices written to out[0..k), padded with -1.
+__device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int k, uint32_t* hist,
+                                          int* __restrict__ out) {
   const int lane = (int)lane_id();
-  const int bi = i >> 6;  // own block (B = 64)
-  const int n_cand = bi + 1;
-  if (n_cand <= k) {  // dense: every visible block
-    for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
-    return;
-  }
-  // ---- max pooling into order keys (forced blocks get the top key); four
-  // 512-byte row segments are loaded before any is used
-  float carry = -INFINITY;  // S^shared[4*base - 1] for the next chunk's lane 0
-  for (int base0 = 0; base0 < n_cand; base0 += 128) {
-    float4 vv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = base0 + 32 * u + lane;
-      const int j0 = 4 * b;
-      float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      if (b < n_cand) {
-        if (j0 + 3 < nv) {
-          v = __ldg(reinterpret_cast<const float4*>(row + j0));
-        } else {
-          if (j0 + 0 < nv) v.x = row[j0 + 0];
-          if (j0 + 1 < nv) v.y = row[j0 + 1];
-          if (j0 + 2 < nv) v.z = row[j0 + 2];
-        }
-      }
-      vv[u] = v;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = base0 + 32 * u + lane;
-      const float4 v = vv[u];
-      // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
-      float prev = __shfl_up_sync(0xFFFFFFFFu, v.w, 1);
-      if (lane == 0) prev = carry;
-      carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
-      if (b < n_cand) {
-        const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
-        const bool forced = b < n_init || b > bi - n_local;
-        keys[b] = forced ? kForcedKey : float_key(m);
-      }
-    }
-  }
-  __syncwarp();
   // ---- radix select of the k-th largest key
   uint32_t prefix = 0, pmask = 0;
   int remaining = k;
@@ -143,6 +97,98 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
   }
   for (int x = written + lane; x < k; x += 32) out[x] = -1;
   __syncwarp();
+}
+
+// Select for one row.  `row` holds S^shared[j] for j < nv (entries at
+// j >= nv may be garbage and are never used; reads stay below 4*(bi+1)).
+// `keys` is per-warp shared scratch of >= bi+1 words, `hist` 256 words.
+// Writes k indices (ascending, -1 padded) to `out`.
+__device__ __forceinline__ void select_row_warp(const float* __restrict__ row, int nv, int i,
+                                                int n_init, int n_local, int k, uint32_t* keys,
+                                                uint32_t* hist, int* __restrict__ out) {
+  const int lane = (int)lane_id();
+  const int bi = i >> 6;  // own block (B = 64)
+  const int n_cand = bi + 1;
+  if (n_cand <= k) {  // dense: every visible block
+    for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
+    return;
+  }
+  // ---- max pooling into order keys (forced blocks get the top key); four
+  // 512-byte row segments are loaded before any is used
+  float carry = -INFINITY;  // S^shared[4*base - 1] for the next chunk's lane 0
+  for (int base0 = 0; base0 < n_cand; base0 += 128) {
+    float4 vv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = base0 + 32 * u + lane;
+      const int j0 = 4 * b;
+      float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (b < n_cand) {
+        if (j0 + 3 < nv) {
+          v = __ldg(reinterpret_cast<const float4*>(row + j0));
+        } else {
+          if (j0 + 0 < nv) v.x = row[j0 + 0];
+          if (j0 + 1 < nv) v.y = row[j0 + 1];
+          if (j0 + 2 < nv) v.z = row[j0 + 2];
+        }
+      }
+      vv[u] = v;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = base0 + 32 * u + lane;
+      const float4 v = vv[u];
+      // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
+      float prev = __shfl_up_sync(0xFFFFFFFFu, v.w, 1);
+      if (lane == 0) prev = carry;
+      carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
+      if (b < n_cand) {
+        const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
+        const bool forced = b < n_init || b > bi - n_local;
+        keys[b] = forced ? kForcedKey : float_key(m);
+      }
+    }
+  }
+  __syncwarp();
+  topk_warp(keys, n_cand, k, hist, out);
+}
+
+// Select for one row from precomputed block scores S^cmp[b] (b < i/B; the own
+// block is always local, so its entry is not read).
+__device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__ cmp, int i,
+                                                       int n_init, int n_local, int k,
+                                                       uint32_t* keys, uint32_t* hist,
+                                                       int* __restrict__ out) {
+  const int lane = (int)lane_id();
+  const int bi = i >> 6;
+  const int n_cand = bi + 1;
+  if (n_cand <= k) {
+    for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
+    return;
+  }
+  for (int base = 0; base < n_cand; base += 128) {
+    float4 vv;
+    const int b0 = base + 4 * lane;
+    if (b0 + 3 < bi) {
+      vv = __ldg(reinterpret_cast<const float4*>(cmp + b0));
+    } else {
+      vv.x = b0 + 0 < bi ? cmp[b0 + 0] : -INFINITY;
+      vv.y = b0 + 1 < bi ? cmp[b0 + 1] : -INFINITY;
+      vv.z = b0 + 2 < bi ? cmp[b0 + 2] : -INFINITY;
+      vv.w = b0 + 3 < bi ? cmp[b0 + 3] : -INFINITY;
+    }
+    const float v4[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + u;
+      if (b < n_cand) {
+        const bool forced = b < n_init || b > bi - n_local;
+        keys[b] = forced ? kForcedKey : float_key(v4[u]);
+      }
+    }
+  }
+  __syncwarp();
+  topk_warp(keys, n_cand, k, hist, out);
 }
 
 // Top-k over block keys already in shared memory (keys[0..bi], forced blocks

@@ -22,7 +22,7 @@ SYMBOLS = [
     "infv2_device_status", "infv2_compress_k", "infv2_block_scores", "infv2_select_topk",
     "infv2_sparse_attn", "infv2_dense_attn", "infv2_prefill_workspace_size", "infv2_prefill",
     "infv2_decode_workspace_size", "infv2_decode", "infv2_select_blocks_noalloc",
-    "infv2_selftest_timeout",
+    "infv2_selftest_timeout", "infv2_block_scores_pooled", "infv2_select_topk_pooled",
 ]
 
 
@@ -62,6 +62,8 @@ def lib():
         L.infv2_compress_k.argtypes = [P, vp, i, vp, vp]
         L.infv2_block_scores.argtypes = [P, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk.argtypes = [P, vp, i, i, i, i, vp, vp]
+        L.infv2_block_scores_pooled.argtypes = [P, vp, vp, i, i, i, vp, i, vp]
+        L.infv2_select_topk_pooled.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_sparse_attn.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
         L.infv2_dense_attn.argtypes = [P, vp, vp, vp, i, vp, vp, vp]
         L.infv2_prefill_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
@@ -163,6 +165,33 @@ def infv2_select_topk(p: Params, s_shared, ld: int, n: int, q_begin: int, q_len:
         idx = torch.full((p.h_kv, n, p.k), -2, dtype=torch.int32, device=s_shared.device)
     _check(lib().infv2_select_topk(ctypes.byref(p), _ptr(s_shared), ld, n, q_begin, q_len,
                                    _ptr(idx), _stream(stream)), "infv2_select_topk")
+    return idx
+
+
+def cmp_ld(n: int) -> int:
+    """Row pitch (floats) of S^cmp for an n-token sequence: blocks rounded to 32."""
+    return ((n + 63) // 64 + 31) // 32 * 32
+
+
+def infv2_block_scores_pooled(p: Params, q, kc1, n: int, q_begin: int, q_len: int, s_cmp=None,
+                              ld_cmp: int | None = None, stream=None):
+    ld_cmp = cmp_ld(n) if ld_cmp is None else ld_cmp
+    if s_cmp is None:
+        s_cmp = torch.zeros((p.h_kv, q_len, ld_cmp), dtype=torch.float32, device=q.device)
+    _check(lib().infv2_block_scores_pooled(ctypes.byref(p), _ptr(q),
+                                           _ptr(kc1) if kc1.numel() else None, n, q_begin,
+                                           q_len, _ptr(s_cmp), ld_cmp, _stream(stream)),
+           "infv2_block_scores_pooled")
+    return s_cmp
+
+
+def infv2_select_topk_pooled(p: Params, s_cmp, ld_cmp: int, n: int, q_begin: int, q_len: int,
+                             idx=None, stream=None):
+    if idx is None:
+        idx = torch.full((p.h_kv, n, p.k), -2, dtype=torch.int32, device=s_cmp.device)
+    _check(lib().infv2_select_topk_pooled(ctypes.byref(p), _ptr(s_cmp), ld_cmp, n, q_begin, q_len,
+                                          _ptr(idx), _stream(stream)),
+           "infv2_select_topk_pooled")
     return idx
 
 
