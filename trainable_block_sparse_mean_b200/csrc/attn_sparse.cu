@@ -274,29 +274,27 @@ __global__ void __launch_bounds__(160, 2)
         sc[1][x] += sd[1][x];
       }
       // ---- causal mask (only a block reaching past the query) and online
-      // softmax with a lazily raised reference max (rows gid and gid+8)
+      // softmax with a lazily raised reference max (rows gid and gid+8).  The
+      // max is taken on the unscaled scores (scale > 0) and the scale is folded
+      // into the exponent argument: p = 2^(s*c - ref), one packed FMA per pair.
       const int t0 = 64 * b + kb;
-      float z[2][4];
-      if (64 * b + 63 <= pos) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) z[nt][e2] = sc[nt][e2] * c;
-      } else {
+      if (64 * b + 63 > pos) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const int t = t0 + nt * 8 + 2 * tig + (e2 & 1);
-            z[nt][e2] = t <= pos ? sc[nt][e2] * c : -INFINITY;
+            if (t > pos) sc[nt][e2] = -INFINITY;
           }
       }
-      float mx0 = fmaxf(fmaxf(z[0][0], z[0][1]), fmaxf(z[1][0], z[1][1]));
-      float mx1 = fmaxf(fmaxf(z[0][2], z[0][3]), fmaxf(z[1][2], z[1][3]));
+      float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+      float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
+      mx0 *= c;
+      mx1 *= c;
       const bool raise = mx0 > m0 + kRescaleSlack || mx1 > m1 + kRescaleSlack;
       if (__any_sync(0xFFFFFFFFu, raise)) {
         const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
@@ -314,15 +312,18 @@ __global__ void __launch_bounds__(160, 2)
           o[nt][3] *= al1;
         }
       }
-      const float ref0 = m0 == -INFINITY ? 0.f : m0;
-      const float ref1 = m1 == -INFINITY ? 0.f : m1;
+      const float2 cpair = make_float2(c, c);
+      const float2 nr0 = make_float2(m0 == -INFINITY ? 0.f : -m0, m0 == -INFINITY ? 0.f : -m0);
+      const float2 nr1 = make_float2(m1 == -INFINITY ? 0.f : -m1, m1 == -INFINITY ? 0.f : -m1);
       float p[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        p[nt][0] = fast_exp2(z[nt][0] - ref0);
-        p[nt][1] = fast_exp2(z[nt][1] - ref0);
-        p[nt][2] = fast_exp2(z[nt][2] - ref1);
-        p[nt][3] = fast_exp2(z[nt][3] - ref1);
+        const float2 x01 = ffma2(make_float2(sc[nt][0], sc[nt][1]), cpair, nr0);
+        const float2 x23 = ffma2(make_float2(sc[nt][2], sc[nt][3]), cpair, nr1);
+        p[nt][0] = fast_exp2(x01.x);
+        p[nt][1] = fast_exp2(x01.y);
+        p[nt][2] = fast_exp2(x23.x);
+        p[nt][3] = fast_exp2(x23.y);
       }
       l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
       l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);

@@ -231,6 +231,45 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction per two
+// lanes' worth of FMA / ADD, each half rounded exactly like its scalar form.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// exp2_fma on a pair, with the packed instructions (same split and polynomial).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  const float2 sh = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, sh);
+  const float2 nn = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 r = ffma2(nn, make_float2(-1.0f, -1.0f), x);
+  float2 p = make_float2(1.32764666e-3f, 1.32764666e-3f);
+  p = ffma2(p, r, make_float2(9.67554096e-3f, 9.67554096e-3f));
+  p = ffma2(p, r, make_float2(5.55071346e-2f, 5.55071346e-2f));
+  p = ffma2(p, r, make_float2(2.40221202e-1f, 2.40221202e-1f));
+  p = ffma2(p, r, make_float2(6.93146944e-1f, 6.93146944e-1f));
+  p = ffma2(p, r, make_float2(1.00000012f, 1.00000012f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -241,14 +241,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           vmax = cm;
         }
         if (vmax != -INFINITY) {
+          // packed pairs: exponent arguments and partial sums two at a time;
+          // a quarter of the exponentials on the FMA pipe
           const float mneg = -vmax * c;
-          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+          const float2 cc = make_float2(c, c), mm = make_float2(mneg, mneg);
+          float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = fmaf(v[e], c, mneg);
-            ps[e & 3] += (e & 3) == 3 ? exp2_fma(x) : fast_exp2(x);
+          for (int e = 0; e < 32; e += 4) {
+            const float2 x01 = ffma2(make_float2(v[e], v[e + 1]), cc, mm);
+            const float2 x23 = ffma2(make_float2(v[e + 2], v[e + 3]), cc, mm);
+            acc01 = fadd2(acc01, make_float2(fast_exp2(x01.x), fast_exp2(x01.y)));
+            acc23 = fadd2(acc23, (e & 4) ? exp2_fma2(x23)
+                                         : make_float2(fast_exp2(x23.x), fast_exp2(x23.y)));
           }
-          l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          l += (acc01.x + acc01.y) + (acc23.x + acc23.y);
         }
         if (it == n_kt - 1) {
           // merge the column groups' statistics of row r
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (mx != -INFINITY) L += s_part[(x * 128 + r) * 2 + 1] * fast_exp2((mx - M) * c);
             }
             const float lse2 = L > 0.f ? M * c + __log2f(L) : -INFINITY;
-            s_lse2[r] = lse2;
+            s_lse2[r] = -lse2;  // stored negated: pass 2 adds it
             if (a.score_lse && i_r <= i_last)
               a.score_lse[(size_t)(g * G + r % G) * a.q_len + (i_r - a.q_begin)] = lse2 * kLn2;
           }
@@ -287,22 +293,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < TPG; ++t) {
           const int tq = cg * TPG + t;
           const int i = i0 + tq;
-          float ps[4] = {0.f, 0.f, 0.f, 0.f};
+          float ssum;
           if constexpr (G >= 4) {
+            // packed pairs; heads 4*h4 .. 4*h4+3 of the token; pairs 3 and 7
+            // of the token's G/2 head pairs (a quarter of G = 8, 16) take the
+            // FMA-pipe exponential
+            const float2 cc = make_float2(c, c);
+            float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int h4 = 0; h4 < G / 4; ++h4) {
-              const float4 L4 = lse4[(t * G) / 4 + h4];  // broadcast read
-              ps[0] += fast_exp2(fmaf(v[t * G + 4 * h4 + 0], c, -L4.x));
-              ps[1] += fast_exp2(fmaf(v[t * G + 4 * h4 + 1], c, -L4.y));
-              ps[2] += fast_exp2(fmaf(v[t * G + 4 * h4 + 2], c, -L4.z));
-              ps[3] += exp2_fma(fmaf(v[t * G + 4 * h4 + 3], c, -L4.w));
+              const float4 L4 = lse4[(t * G) / 4 + h4];  // broadcast read of -lse2
+              const float2 x01 = ffma2(make_float2(v[t * G + 4 * h4 + 0], v[t * G + 4 * h4 + 1]), cc,
+                                       make_float2(L4.x, L4.y));
+              const float2 x23 = ffma2(make_float2(v[t * G + 4 * h4 + 2], v[t * G + 4 * h4 + 3]), cc,
+                                       make_float2(L4.z, L4.w));
+              acc01 = fadd2(acc01, make_float2(fast_exp2(x01.x), fast_exp2(x01.y)));
+              acc23 = fadd2(acc23, (h4 & 1) ? exp2_fma2(x23)
+                                            : make_float2(fast_exp2(x23.x), fast_exp2(x23.y)));
             }
+            ssum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
           } else {
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int hh = 0; hh < G; ++hh)
-              ps[hh] += fast_exp2(fmaf(v[t * G + hh], c, -s_lse2[tq * G + hh]));
+              ps[hh] += fast_exp2(fmaf(v[t * G + hh], c, s_lse2[tq * G + hh]));
+            ssum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
           }
-          const float ssum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
           const bool vis = i <= i_last && j < visible_kernels(i, 32, 16);
           if constexpr (POOL) {
             pv[t] = vis ? ssum : -INFINITY;
