@@ -32,15 +32,16 @@ class Params(ctypes.Structure):
                 ("pool_l", ctypes.c_int), ("pool_s", ctypes.c_int),
                 ("n_init", ctypes.c_int), ("n_local", ctypes.c_int), ("k", ctypes.c_int),
                 ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("d", ctypes.c_int),
-                ("scale", ctypes.c_double), ("pool_rule", ctypes.c_int)]
+                ("scale", ctypes.c_double), ("pool_rule", ctypes.c_int),
+                ("lse_approx", ctypes.c_int)]
 
 
-def params(shape, scale=None, pool_rule=0) -> Params:
+def params(shape, scale=None, pool_rule=0, lse_approx=0) -> Params:
     """Oracle parameters from a synth.Shape (scale defaults to 1/sqrt(d))."""
     sc = 1.0 / np.sqrt(shape.d) if scale is None else float(scale)
     return Params(shape.B, shape.l_c1, shape.s_c1, shape.pool_l, shape.pool_s,
                   shape.n_init, shape.n_local, shape.k, shape.h_q, shape.h_kv, shape.d,
-                  sc, pool_rule)
+                  sc, pool_rule, lse_approx)
 
 
 def _declare(L):
@@ -53,6 +54,11 @@ def _declare(L):
     L.orc_num_kernels.argtypes = [P, i]
     L.orc_visible_kernels.argtypes = [P, i]
     L.orc_compress_k.argtypes = [P, vp, i, vp]
+    L.orc_num_coarse_kernels.argtypes = [P, i]
+    L.orc_visible_coarse_kernels.argtypes = [P, i]
+    L.orc_compress_k2.argtypes = [P, vp, i, vp]
+    L.orc_coarse_lse_row.argtypes = [P, vp, vp, i, i, vp]
+    L.orc_shared_scores_row_lse.argtypes = [P, vp, vp, i, i, vp, vp, vp]
     L.orc_shared_scores_row.argtypes = [P, vp, vp, i, i, vp, vp]
     L.orc_block_scores_row.argtypes = [P, vp, i, i, vp]
     L.orc_select_row.argtypes = [P, vp, i, vp]
@@ -128,6 +134,45 @@ def compress_k(p: Params, k: np.ndarray) -> np.ndarray:
     out = np.zeros((max(num_kernels(p, n), 0), p.h_kv, p.d), np.uint16)
     _L().orc_compress_k(ctypes.byref(p), _ptr(k), n, _ptr(out))
     return out
+
+
+def num_coarse_kernels(p: Params, n: int) -> int:
+    return _L().orc_num_coarse_kernels(ctypes.byref(p), n)
+
+
+def visible_coarse_kernels(p: Params, i: int) -> int:
+    return _L().orc_visible_coarse_kernels(ctypes.byref(p), i)
+
+
+def compress_k2(p: Params, k: np.ndarray) -> np.ndarray:
+    """Coarse kernels K^C2 of the LSE approximation (l_C2 = 4 l_C1, s_C2 = 4 s_C1)."""
+    k = _c(k, np.uint16)
+    n = k.shape[0]
+    out = np.zeros((max(num_coarse_kernels(p, n), 0), p.h_kv, p.d), np.uint16)
+    _L().orc_compress_k2(ctypes.byref(p), _ptr(k), n, _ptr(out))
+    return out
+
+
+def coarse_lse_row(p: Params, q, kc2, i: int, g: int):
+    """Approximate per-head LSE of row i (None when no coarse kernel is visible)."""
+    q = _c(q, np.uint16)
+    kc2 = _c(kc2, np.uint16)
+    out = np.zeros(p.h_q // p.h_kv, np.float64)
+    ok = _L().orc_coarse_lse_row(ctypes.byref(p), _ptr(q), _ptr(kc2), i, g, _ptr(out))
+    return out if ok else None
+
+
+def shared_scores_row_lse(p: Params, q, kc1, i: int, g: int, lse_in=None):
+    """S^shared of row i normalised by the given per-head LSE (exact when None)."""
+    q = _c(q, np.uint16)
+    kc1 = _c(kc1, np.uint16)
+    nv = visible_kernels(p, i)
+    out = np.zeros(max(nv, 1), np.float64)
+    lse = np.zeros(p.h_q // p.h_kv, np.float64)
+    li = None if lse_in is None else _c(np.asarray(lse_in, np.float64), np.float64)
+    _L().orc_shared_scores_row_lse(ctypes.byref(p), _ptr(q), _ptr(kc1), i, g,
+                                   None if li is None else _ptr(li), _ptr(out), _ptr(lse))
+    return out[:nv], lse
 
 
 def shared_scores_row(p: Params, q, kc1, i: int, g: int):

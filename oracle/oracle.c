@@ -17,6 +17,9 @@
  *    infinite score; sequences no longer than k blocks use dense attention.
  *  - arXiv 2509.24663 summary, Appendix A: attention of each query over the
  *    visible tokens of its selected blocks, returning O and the log-sum-exp.
+ *  - same notes, key design 4, and the blog's efficient top-k: the optional
+ *    LSE approximation estimates each head's log-sum-exp from coarser kernels
+ *    K^C2 (l_C2 = 4 l_C1, s_C2 = 4 s_C1) instead of the K^C1 kernels.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - scale 1/sqrt(d) on the score logits and the attention logits (parameter);
@@ -24,7 +27,12 @@
  *  - K^C1 is a bf16 tensor: the exact mean rounded once, nearest-even;
  *  - the local set is {b_i - n_local + 1 .. b_i} (own block included);
  *  - k counts every selected block, init and local included;
- *  - equal block scores are ordered by lower block index.
+ *  - equal block scores are ordered by lower block index;
+ *  - LSE approximation (optional): K^C2 is rounded to bf16 like K^C1, a coarse
+ *    kernel is visible under the same rule, the estimate is the log-sum-exp
+ *    over the visible coarse kernels plus log(s_C2 / s_C1) (each coarse kernel
+ *    stands for that many stage-1 kernels), and a row that sees no coarse
+ *    kernel keeps the exact log-sum-exp.
  */
 #include <math.h>
 #include <stdint.h>
@@ -46,6 +54,7 @@ typedef struct {
     int h_q, h_kv, d;
     double scale; /* logit scale */
     int pool_rule;/* 0: kernels intersecting the block; 1: literal window */
+    int lse_approx;/* 1: pass-1 log-sum-exp estimated from the coarse kernels K^C2 */
 } orc_params;
 
 int orc_num_threads(void) {
@@ -116,11 +125,71 @@ void orc_compress_k(const orc_params* p, const uint16_t* k, int n, uint16_t* kc1
             }
 }
 
+/* The coarse kernels of the LSE approximation: the stage-1 definitions with
+ * l_C2 = 4 l_C1 and s_C2 = 4 s_C1. */
+static orc_params coarse_params(const orc_params* p) {
+    orc_params c = *p;
+    c.l_c1 = 4 * p->l_c1;
+    c.s_c1 = 4 * p->s_c1;
+    return c;
+}
+
+int orc_num_coarse_kernels(const orc_params* p, int n) {
+    orc_params c = coarse_params(p);
+    return orc_num_kernels(&c, n);
+}
+
+int orc_visible_coarse_kernels(const orc_params* p, int i) {
+    orc_params c = coarse_params(p);
+    return orc_visible_kernels(&c, i);
+}
+
+/* K^C2[c, g, :] = bf16(mean of K over the coarse kernel's l_C2 tokens). */
+void orc_compress_k2(const orc_params* p, const uint16_t* k, int n, uint16_t* kc2) {
+    orc_params c = coarse_params(p);
+    orc_compress_k(&c, k, n, kc2);
+}
+
+/* Natural log-sum-exp over j < nv of scale * q_{i,h} . K_j (K = kc, [*, h_kv, d]). */
+static double lse_over(const orc_params* p, const uint16_t* q, const uint16_t* kc, int nv,
+                       int i, int h, int g, double* z) {
+    const uint16_t* qr = q + ((size_t)i * p->h_q + h) * p->d;
+    double m = -INFINITY;
+    for (int j = 0; j < nv; ++j) {
+        const uint16_t* kr = kc + ((size_t)j * p->h_kv + g) * p->d;
+        double dot = 0.0;
+        for (int c = 0; c < p->d; ++c) dot += bf16_value(qr[c]) * bf16_value(kr[c]);
+        z[j] = p->scale * dot;
+        if (z[j] > m) m = z[j];
+    }
+    if (nv == 0) return -INFINITY;
+    double s = 0.0;
+    for (int j = 0; j < nv; ++j) s += exp(z[j] - m);
+    return m + log(s);
+}
+
+/* LSE approximation for row i, group g: lse_h ~= log sum over the visible
+ * coarse kernels of exp(scale * q_{i,h} . K^C2_c) + log(s_C2 / s_C1).
+ * Returns 0 (and writes nothing) when the row sees no coarse kernel. */
+int orc_coarse_lse_row(const orc_params* p, const uint16_t* q, const uint16_t* kc2, int i, int g,
+                       double* lse_out) {
+    int nv2 = orc_visible_coarse_kernels(p, i);
+    if (nv2 == 0) return 0;
+    int G = p->h_q / p->h_kv;
+    double* z = (double*)malloc(sizeof(double) * nv2);
+    for (int hh = 0; hh < G; ++hh)
+        lse_out[hh] = lse_over(p, q, kc2, nv2, i, g * G + hh, g, z) + log(4.0);
+    free(z);
+    return 1;
+}
+
 /* Stage 2 for one query row i and group g: S^shared[j] = sum over the group's
  * heads h of softmax_j(scale * q_{i,h} . K^C1_j), j over the visible kernels.
- * lse_out (nullable, G entries) receives each head's natural log-sum-exp. */
-void orc_shared_scores_row(const orc_params* p, const uint16_t* q, const uint16_t* kc1,
-                           int i, int g, double* out, double* lse_out) {
+ * The softmax is normalised by lse_in[hh] when given (the LSE approximation),
+ * else by the exact log-sum-exp over the visible kernels.  lse_out (nullable,
+ * G entries) receives the log-sum-exp used. */
+void orc_shared_scores_row_lse(const orc_params* p, const uint16_t* q, const uint16_t* kc1,
+                               int i, int g, const double* lse_in, double* out, double* lse_out) {
     int nv = orc_visible_kernels(p, i);
     int G = p->h_q / p->h_kv;
     for (int j = 0; j < nv; ++j) out[j] = 0.0;
@@ -131,22 +200,17 @@ void orc_shared_scores_row(const orc_params* p, const uint16_t* q, const uint16_
     double* z = (double*)malloc(sizeof(double) * nv);
     for (int hh = 0; hh < G; ++hh) {
         int h = g * G + hh;
-        const uint16_t* qr = q + ((size_t)i * p->h_q + h) * p->d;
-        double m = -INFINITY;
-        for (int j = 0; j < nv; ++j) {
-            const uint16_t* kr = kc1 + ((size_t)j * p->h_kv + g) * p->d;
-            double dot = 0.0;
-            for (int c = 0; c < p->d; ++c) dot += bf16_value(qr[c]) * bf16_value(kr[c]);
-            z[j] = p->scale * dot;
-            if (z[j] > m) m = z[j];
-        }
-        double s = 0.0;
-        for (int j = 0; j < nv; ++j) s += exp(z[j] - m);
-        double lse = m + log(s);
+        double lse = lse_over(p, q, kc1, nv, i, h, g, z);
+        if (lse_in) lse = lse_in[hh];
         for (int j = 0; j < nv; ++j) out[j] += exp(z[j] - lse);
         if (lse_out) lse_out[hh] = lse;
     }
     free(z);
+}
+
+void orc_shared_scores_row(const orc_params* p, const uint16_t* q, const uint16_t* kc1,
+                           int i, int g, double* out, double* lse_out) {
+    orc_shared_scores_row_lse(p, q, kc1, i, g, NULL, out, lse_out);
 }
 
 /* Does stage-1 kernel j belong to block b's pooling window? */
@@ -273,6 +337,12 @@ void orc_prefill_rows(const orc_params* p, const uint16_t* q, const uint16_t* k,
     int dense = n <= p->k * p->B;
     uint16_t* kc1 = (uint16_t*)malloc(sizeof(uint16_t) * ((size_t)nc * p->h_kv * p->d + 1));
     orc_compress_k(p, k, n, kc1);
+    uint16_t* kc2 = NULL;
+    if (p->lse_approx) {
+        int nc2 = orc_num_coarse_kernels(p, n);
+        kc2 = (uint16_t*)malloc(sizeof(uint16_t) * ((size_t)nc2 * p->h_kv * p->d + 1));
+        orc_compress_k2(p, k, n, kc2);
+    }
     int need_scores = !dense || cmp_out || shared_out || score_lse_out;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < nrows; ++r) {
@@ -285,7 +355,9 @@ void orc_prefill_rows(const orc_params* p, const uint16_t* q, const uint16_t* k,
             int* idx = idx_out + ((size_t)r * p->h_kv + g) * p->k;
             double* slse = score_lse_out ? score_lse_out + (size_t)r * p->h_q + g * G : NULL;
             if (need_scores) {
-                orc_shared_scores_row(p, q, kc1, i, g, shared, slse);
+                double approx[64];  /* G <= 64 */
+                int use = kc2 && orc_coarse_lse_row(p, q, kc2, i, g, approx);
+                orc_shared_scores_row_lse(p, q, kc1, i, g, use ? approx : NULL, shared, slse);
                 orc_block_scores_row(p, shared, nv, i, cmp);
             }
             if (shared_out) {
@@ -312,6 +384,7 @@ void orc_prefill_rows(const orc_params* p, const uint16_t* q, const uint16_t* k,
         free(shared);
     }
     free(kc1);
+    free(kc2);
 }
 
 /* Selection alone, from given S^shared rows (values already in the precision

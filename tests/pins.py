@@ -136,6 +136,85 @@ def pin_visibility():
         assert oracle.visible_kernels(p, i) == want, (i,)
 
 
+def pin_coarse_kernels_bruteforce():
+    """LSE approximation: K^C2 is the bf16 mean over l_C2 = 4 l_C1 = 128 tokens at
+    stride s_C2 = 4 s_C1 = 64, visible to query i when its last token is <= i."""
+    sh = _shape(n=300, h_q=2, h_kv=2, d=8)
+    p = oracle.params(sh)
+    for n in range(0, 400, 7):
+        assert oracle.num_coarse_kernels(p, n) == sum(1 for c in range(n) if 64 * c + 128 <= n), (n,)
+    for i in range(0, 400, 3):
+        assert oracle.visible_coarse_kernels(p, i) == sum(1 for c in range(i + 1) if 64 * c + 127 <= i), (i,)
+    rng = np.random.default_rng(12)
+    k = _bf16(rng.standard_normal((300, 2, 8)).astype(np.float32) * 3)
+    kv = _f64(k)
+    kc2 = _f64(oracle.compress_k2(p, k))
+    assert kc2.shape == ((300 - 128) // 64 + 1, 2, 8), kc2.shape
+    for c in range(kc2.shape[0]):
+        for g in range(2):
+            for e in range(8):
+                s_ = sum(Fraction(float(kv[t, g, e])) for t in range(64 * c, 64 * c + 128))
+                want = _rne_bf16_fraction(s_ / 128)
+                assert kc2[c, g, e] == want, (c, g, e, kc2[c, g, e], want)
+
+
+def pin_coarse_lse_closed_forms():
+    """Constant keys: every logit is z0, so the estimate is z0 + log(nv2) + log 4 and
+    each normalised score is exp(z0 - estimate) = 1 / (4 nv2).  Two visible coarse
+    kernels: the estimate is max + log(1 + exp(-|D|)) + log 4."""
+    sh = _shape(n=512, h_q=4, h_kv=2, d=8)
+    p = oracle.params(sh)
+    rng = np.random.default_rng(21)
+    q = _bf16(rng.standard_normal((512, 4, 8)))
+    k = _bf16(np.broadcast_to(rng.standard_normal((1, 2, 8)), (512, 2, 8)))
+    kc1, kc2 = oracle.compress_k(p, k), oracle.compress_k2(p, k)
+    qf, kf = _f64(q), _f64(k)
+    for i in (127, 191, 300, 511):
+        nv2 = (i - 127) // 64 + 1
+        nv1 = (i - 31) // 16 + 1
+        for g in range(2):
+            lse = oracle.coarse_lse_row(p, q, kc2, i, g)
+            assert lse is not None, (i, g)
+            for hh in range(2):
+                z0 = float(qf[i, g * 2 + hh] @ kf[0, g]) / np.sqrt(8)
+                assert abs(lse[hh] - (z0 + np.log(nv2) + np.log(4.0))) < 1e-12, (i, g, hh)
+            s_, used = oracle.shared_scores_row_lse(p, q, kc1, i, g, lse)
+            assert np.allclose(used, lse, rtol=0, atol=0)
+            assert np.allclose(s_, 2.0 / (4 * nv2), rtol=1e-12, atol=0), (i, s_[:3])
+            assert len(s_) == nv1
+    sh, data = _small_problem(n=256, h_q=4, h_kv=2, d=16, seed=13)
+    p = oracle.params(sh)
+    kc2 = oracle.compress_k2(p, data["k"])
+    qf, K2 = _f64(data["q"]), _f64(kc2)
+    for g in range(2):
+        lse = oracle.coarse_lse_row(p, data["q"], kc2, 191, g)   # coarse kernels 0 and 1
+        assert lse is not None
+        for hh in range(2):
+            z = [float(qf[191, g * 2 + hh] @ K2[c, g]) / 4.0 for c in (0, 1)]
+            want = max(z) + np.log1p(np.exp(-abs(z[0] - z[1]))) + np.log(4.0)
+            assert abs(lse[hh] - want) < 1e-12, (g, hh, lse[hh], want)
+        assert oracle.coarse_lse_row(p, data["q"], kc2, 126, g) is None
+
+
+def pin_coarse_lse_only_where_a_coarse_kernel_is_visible():
+    """With the approximation on, rows that see no coarse kernel keep the exact
+    log-sum-exp and scores; later rows use the estimate."""
+    sh, data = _small_problem(n=400, h_q=4, h_kv=2, d=16, seed=17)
+    pe, pa = oracle.params(sh), oracle.params(sh, lse_approx=1)
+    rows = np.array([31, 64, 126, 127, 250, 399], np.int32)
+    ex = oracle.prefill_rows(pe, data["q"], data["k"], data["v"], rows, want_shared=True, want_score_lse=True)
+    ap = oracle.prefill_rows(pa, data["q"], data["k"], data["v"], rows, want_shared=True, want_score_lse=True)
+    kc2 = oracle.compress_k2(pa, data["k"])
+    for r, i in enumerate(rows):
+        if i < 127:
+            assert np.array_equal(ex["shared"][r], ap["shared"][r]) and np.array_equal(ex["score_lse"][r], ap["score_lse"][r])
+        else:
+            for g in range(2):
+                want = oracle.coarse_lse_row(pa, data["q"], kc2, int(i), g)
+                assert want is not None and np.array_equal(ap["score_lse"][r, g * 2:g * 2 + 2], want)
+            assert not np.array_equal(ex["score_lse"][r], ap["score_lse"][r])
+
+
 # --------------------------------------------------------------------------
 # stage 2: S^C1 softmax and the group sum S^shared
 # --------------------------------------------------------------------------

@@ -15,9 +15,11 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
 MUTANTS = {
     "visibility_off_by_one": ("j * p->s_c1 + p->l_c1 - 1 <= i; ++j", "j * p->s_c1 + p->l_c1 <= i; ++j"),
-    "head_group_mapping": ("int h = g * G + hh;\n        const uint16_t* qr = q + ((size_t)i * p->h_q + h) * p->d;\n        double m = -INFINITY;\n        for (int j = 0;",
-                           "int h = hh * p->h_kv + g;\n        const uint16_t* qr = q + ((size_t)i * p->h_q + h) * p->d;\n        double m = -INFINITY;\n        for (int j = 0;"),
-    "lse_drops_max": ("double lse = m + log(s);", "double lse = log(s);"),
+    "head_group_mapping": ("int h = g * G + hh;\n        double lse = lse_over(", "int h = hh * p->h_kv + g;\n        double lse = lse_over("),
+    "lse_drops_max": ("return m + log(s);", "return log(s);"),
+    "coarse_correction_dropped": ("lse_over(p, q, kc2, nv2, i, g * G + hh, g, z) + log(4.0);", "lse_over(p, q, kc2, nv2, i, g * G + hh, g, z);"),
+    "coarse_stride": ("c.s_c1 = 4 * p->s_c1;", "c.s_c1 = 2 * p->s_c1;"),
+    "coarse_length": ("c.l_c1 = 4 * p->l_c1;", "c.l_c1 = 2 * p->l_c1;"),
     "score_scale_dropped": ("z[j] = p->scale * dot;", "z[j] = dot;"),
     "pool_window_literal_start": ("return k_first <= b_last && k_last >= b_first;", "return k_first >= b_first && k_first <= b_last;"),
     "ties_to_higher_block": ("return (a->b > c->b) - (a->b < c->b);", "return (a->b < c->b) - (a->b > c->b);"),
