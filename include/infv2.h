@@ -70,6 +70,16 @@ enum infv2_status {
  *   scale    logit scale of both the scores and the attention (1/sqrt(d))
  *   window   sliding window (tokens) that the local blocks must cover:
  *            n_local >= ceil(window / B) + 1 is enforced (0 = no window)
+ *   lse_approx  0: exact two-pass scores (default).  1: the LSE
+ *            approximation (paper notes, key design 4; MiniCPM4 blog,
+ *            efficient top-k): pass 1 estimates each head's log-sum-exp from
+ *            coarse kernels K^C2 (l_C2 = 4 l_c1, s_C2 = 4 s_c1) as
+ *            log sum_{visible c} exp(scale q . K^C2_c) + log(s_C2 / s_c1);
+ *            rows that see no coarse kernel keep the exact value.  Used by
+ *            infv2_prefill; infv2_decode (and its workspace query) returns
+ *            INFV2_ERR_UNSUPPORTED when it is set; the stage entry points
+ *            and infv2_select_blocks_noalloc do not read it (the approximate
+ *            scores have their own entry, infv2_block_scores_approx).
  * This build's kernels support d = 128, B = 64, l_c1 = 32, s_c1 = 16,
  * pool_l = 5, pool_s = 4, h_q % h_kv == 0 with G = h_q/h_kv in {1,2,4,8,16},
  * k >= n_init + n_local, n_local >= 1 and k <= 256.  Other values return
@@ -80,10 +90,12 @@ typedef struct infv2_params {
   int h_q, h_kv, d;
   float scale;
   int window;
+  int lse_approx;
 } infv2_params;
 
 /* Fill *p with the paper's hyper-parameters (B=64, l_c1=32, s_c1=16, l=5,
- * s=4, n_init=1, n_local=2, k=64, d=128, scale=1/sqrt(128)) for h_q, h_kv. */
+ * s=4, n_init=1, n_local=2, k=64, d=128, scale=1/sqrt(128)) for h_q, h_kv,
+ * with window 0 and the exact scores (lse_approx 0). */
 void infv2_default_params(infv2_params* p, int h_q, int h_kv);
 
 /* Validate *p against the method and this build.  Returns INFV2_OK,
@@ -109,6 +121,14 @@ int infv2_device_status(infv2_stream_t stream);
 int infv2_compress_k(const infv2_params* p, const void* k, int n, void* kc1,
                      infv2_stream_t stream);
 
+/* Coarse kernels of the LSE approximation (paper notes, key design 4):
+ * K^C2[c, g, :] = bf16 round-to-nearest-even of the exact mean of K[t, g, :]
+ * over t = c*4*s_c1 .. c*4*s_c1 + 4*l_c1 - 1 (128 tokens at stride 64).
+ *   k    bf16 [n, h_kv, d];  kc2  bf16 [num_coarse_kernels(n), h_kv, d] (output)
+ * num_coarse_kernels(n) = n >= 4*l_c1 ? (n - 4*l_c1) / (4*s_c1) + 1 : 0. */
+int infv2_compress_k2(const infv2_params* p, const void* k, int n, void* kc2,
+                      infv2_stream_t stream);
+
 /* Stage 2, fused two-pass scores (paper notes, key design 4; arXiv summary,
  * section 3): for query rows i in [q_begin, q_begin + q_len) of an n-token
  * sequence and kv head g, with J(i) the kernels j where j*s_c1 + l_c1 - 1 <= i,
@@ -122,6 +142,17 @@ int infv2_compress_k(const infv2_params* p, const void* k, int n, void* kc1,
 int infv2_block_scores(const infv2_params* p, const void* q, const void* kc1, int n, int q_begin,
                        int q_len, float* s_shared, int ld, float* score_lse,
                        infv2_stream_t stream);
+
+/* infv2_block_scores with the LSE approximation: lse_h is the coarse estimate
+ * of the lse_approx parameter (whatever p->lse_approx holds) for rows that see
+ * a coarse kernel (i >= 4*l_c1 - 1), the exact value for the others.  Pass 1
+ * then runs over the coarse kernels, a quarter as many as pass 2's.
+ *   kc2  bf16 [num_coarse_kernels(n), h_kv, d] from infv2_compress_k2
+ * Other arguments and outputs as infv2_block_scores (score_lse receives the
+ * log-sum-exp used). */
+int infv2_block_scores_approx(const infv2_params* p, const void* q, const void* kc1,
+                              const void* kc2, int n, int q_begin, int q_len, float* s_shared,
+                              int ld, float* score_lse, infv2_stream_t stream);
 
 /* Stages 3-4 (paper notes, key designs 2-3; MiniCPM4 blog, semantic kernels):
  * for each row i in [q_begin, q_begin + q_len) and kv head g, block scores

@@ -111,4 +111,17 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,
                           None, None) == infv2.OK
     assert L.infv2_selftest_timeout(0, None) == infv2.ERR_INVALID_ARG
+    # the LSE approximation flag: 0 or 1; decode does not take it
+    assert p.lse_approx == 0
+    pa = infv2.params(32, 2, lse_approx=1)
+    assert L.infv2_check_params(ctypes.byref(pa)) == infv2.OK
+    pa.lse_approx = 2
+    assert L.infv2_check_params(ctypes.byref(pa)) == infv2.ERR_INVALID_ARG
+    pa.lse_approx = 1
+    sz = ctypes.c_size_t()
+    assert L.infv2_decode_workspace_size(ctypes.byref(pa), 4, 4096, ctypes.byref(sz)) == infv2.ERR_UNSUPPORTED
+    assert L.infv2_compress_k2(P, None, 0, None, None) == infv2.OK
+    assert L.infv2_compress_k2(P, None, 200, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_block_scores_approx(P, None, None, None, 100, 50, 60, None, 128, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_prefill_workspace_size(ctypes.byref(pa), (ctypes.c_int * 2)(0, 10000), 1, ctypes.byref(sz)) == infv2.OK
     assert L.infv2_check_params(None) == infv2.ERR_INVALID_ARG

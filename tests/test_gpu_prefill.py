@@ -22,8 +22,9 @@ def _lib():
     infv2.lib()
 
 
-def run_prefill(shape, data, cu):
+def run_prefill(shape, data, cu, lse_approx=0):
     p = infv2.params_of(shape)
+    p.lse_approx = lse_approx
     q, k, v = to_dev(data["q"]), to_dev(data["k"]), to_dev(data["v"])
     T = q.shape[0]
     idx = torch.full((shape.h_kv, T, shape.k), -3, dtype=torch.int32, device="cuda")
@@ -34,9 +35,9 @@ def run_prefill(shape, data, cu):
     return dict(p=p, q=q, k=k, v=v, o=o, idx=idx, lse=lse)
 
 
-def check_sequence(shape, data, dev, off, n, rows, dense, max_bad=0):
+def check_sequence(shape, data, dev, off, n, rows, dense, max_bad=0, lse_approx=0):
     """Compare rows (sequence-local) of one sequence starting at token `off`."""
-    op = oracle.params(shape)
+    op = oracle.params(shape, lse_approx=lse_approx)
     sl = slice(off, off + n)
     ref = oracle.prefill_rows(op, data["q"][sl], data["k"][sl], data["v"][sl], rows, want_cmp=True)
     o_gpu = synth.bf16_to_f32(to_host_bits(dev["o"][sl]))[rows]

@@ -127,13 +127,15 @@ void infv2_default_params(infv2_params* p, int h_q, int h_kv) {
   p->d = 128;
   p->scale = 1.0f / sqrtf(128.0f);
   p->window = 0;
+  p->lse_approx = 0;
 }
 
 int infv2_check_params(const infv2_params* p) {
   if (!p) return INFV2_ERR_INVALID_ARG;
   if (p->B <= 0 || p->l_c1 <= 0 || p->s_c1 <= 0 || p->pool_l <= 0 || p->pool_s <= 0 ||
       p->n_init < 0 || p->n_local < 1 || p->k <= 0 || p->h_q <= 0 || p->h_kv <= 0 || p->d <= 0 ||
-      p->window < 0 || !(p->scale > 0.0f) || !isfinite(p->scale))
+      p->window < 0 || !(p->scale > 0.0f) || !isfinite(p->scale) ||
+      (p->lse_approx != 0 && p->lse_approx != 1))
     return INFV2_ERR_INVALID_ARG;
   if (p->h_q % p->h_kv != 0) return INFV2_ERR_INVALID_ARG;
   if (p->k < p->n_init + p->n_local) return INFV2_ERR_INVALID_ARG;

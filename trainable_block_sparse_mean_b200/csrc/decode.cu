@@ -352,6 +352,7 @@ extern "C" int infv2_decode_workspace_size(const infv2_params* p, int batch, int
                                            size_t* bytes) {
   int st = infv2_check_params(p);
   if (st != INFV2_OK) return st;
+  if (p->lse_approx) return INFV2_ERR_UNSUPPORTED;  // the decode step scores exactly
   if (!bytes || batch < 0 || cap < 0) return INFV2_ERR_INVALID_ARG;
   *bytes = plan_decode(p, batch, cap).total;
   return INFV2_OK;
@@ -363,6 +364,7 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
                             int* idx_out, void* o, float* lse, infv2_stream_t stream) {
   int st = infv2_check_params(p);
   if (st != INFV2_OK) return st;
+  if (p->lse_approx) return INFV2_ERR_UNSUPPORTED;  // the decode step scores exactly
   if (batch < 0 || cap <= 0) return INFV2_ERR_INVALID_ARG;
   if (batch == 0) return INFV2_OK;
   if (!q || !k_new || !v_new || !k_cache || !v_cache || !seqlens || !o) return INFV2_ERR_INVALID_ARG;

@@ -6,9 +6,18 @@ namespace infv2 {
 
 int launch_compress_k(const uint16_t* k, int n, int h_kv, uint16_t* kc1, cudaStream_t st);
 
+// Coarse kernels of the LSE approximation: length 128, stride 64.
+int launch_compress_k2(const uint16_t* k, int n, int h_kv, uint16_t* kc2, cudaStream_t st);
+inline int num_coarse_kernels(int n) { return n >= 128 ? (n - 128) / 64 + 1 : 0; }
+
 int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
                         int q_begin, int q_len, float* s_shared, int ld, float* score_lse,
                         cudaStream_t st);
+
+// Scores with the LSE approximation (pass 1 over K^C2 for rows i >= 127).
+int launch_block_scores_approx(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
+                               const uint16_t* kc2, int n, int q_begin, int q_len,
+                               float* s_shared, int ld, float* score_lse, cudaStream_t st);
 
 int launch_select(const infv2_params* p, const float* s_shared, int ld, int n, int q_begin,
                   int q_len, int* idx, long long idx_hstride, cudaStream_t st);

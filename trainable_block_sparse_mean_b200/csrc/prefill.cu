@@ -15,7 +15,7 @@ constexpr size_t kSharedChunkBytes = size_t(256) << 20;  // S^shared buffer budg
 
 struct PrefillPlan {
   int max_sparse_n = 0;
-  size_t off_kc1 = 0, off_shared = 0, off_idx = 0, total = 0;
+  size_t off_kc1 = 0, off_kc2 = 0, off_shared = 0, off_idx = 0, total = 0;
   int ld = 0, chunk = 0;
 };
 
@@ -36,7 +36,9 @@ int plan_prefill(const infv2_params* p, const int* cu, int batch, PrefillPlan* p
   if (chunk > (size_t)n) chunk = n;
   pl->chunk = (int)chunk;
   pl->off_kc1 = 0;
-  pl->off_shared = round256(nc * p->h_kv * 128 * 2);
+  pl->off_kc2 = round256(nc * p->h_kv * 128 * 2);
+  const size_t nc2 = p->lse_approx ? (size_t)num_coarse_kernels(n) : 0;  // LSE approximation
+  pl->off_shared = pl->off_kc2 + round256(nc2 * p->h_kv * 128 * 2);
   pl->off_idx = pl->off_shared + round256(row_bytes * chunk);
   pl->total = pl->off_idx + round256((size_t)p->h_kv * n * p->k * 4);
   return INFV2_OK;
@@ -94,6 +96,7 @@ extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* kc1 = reinterpret_cast<uint16_t*>(ws + pl.off_kc1);
+  uint16_t* kc2 = reinterpret_cast<uint16_t*>(ws + pl.off_kc2);
   float* s_shared = reinterpret_cast<float*>(ws + pl.off_shared);
   int* idx_ws = reinterpret_cast<int*>(ws + pl.off_idx);
   const uint16_t* qb = static_cast<const uint16_t*>(q);
@@ -116,11 +119,17 @@ extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k
     }
     st = launch_compress_k(ks, n, p->h_kv, kc1, cs);
     if (st != INFV2_OK) return st;
+    if (p->lse_approx) {
+      st = launch_compress_k2(ks, n, p->h_kv, kc2, cs);
+      if (st != INFV2_OK) return st;
+    }
     int* idx = idx_out ? idx_out + off * p->k : idx_ws;
     const long long hstride = idx_out ? T * p->k : (long long)n * p->k;
     for (int q0 = 0; q0 < n; q0 += pl.chunk) {
       const int ql = n - q0 < pl.chunk ? n - q0 : pl.chunk;
-      st = launch_block_scores(p, qs, kc1, n, q0, ql, s_shared, pl.ld, nullptr, cs);
+      st = p->lse_approx
+               ? launch_block_scores_approx(p, qs, kc1, kc2, n, q0, ql, s_shared, pl.ld, nullptr, cs)
+               : launch_block_scores(p, qs, kc1, n, q0, ql, s_shared, pl.ld, nullptr, cs);
       if (st != INFV2_OK) return st;
       st = launch_select(p, s_shared, pl.ld, n, q0, ql, idx, hstride, cs);
       if (st != INFV2_OK) return st;

@@ -40,13 +40,15 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct ScoreArgs {
-  int q_begin, q_len, n_tiles;
+  int q_begin, q_len, n_tiles;   // rows computed by this launch
+  int o_begin, o_len;            // row range of the output buffers (row i at i - o_begin)
+  int approx;                    // 1: pass 1 over the coarse kernels K^C2 (LSE approximation)
   float scale_log2;     // scale * log2(e)
   int ld;
-  float* s_shared;      // [h_kv, q_len, ld]      (unpooled form)
-  float* s_cmp;         // [h_kv, q_len, ld_cmp]  (pooled form: block scores)
+  float* s_shared;      // [h_kv, o_len, ld]      (unpooled form)
+  float* s_cmp;         // [h_kv, o_len, ld_cmp]  (pooled form: block scores)
   int ld_cmp;
-  float* score_lse;     // [h_q, q_len] or null
+  float* score_lse;     // [h_q, o_len] or null
   WaitCtx wait;
 };
 
@@ -68,7 +70,7 @@ struct ScoreSmem {
 template <int G, bool POOL>
 __global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 ScoreArgs a) {
+                 const __grid_constant__ CUtensorMap tm_k2, ScoreArgs a) {
   constexpr int TQ = 128 / G;
   constexpr int TPG = kCols / G > 0 ? kCols / G : 1;  // tokens per column group
   extern __shared__ uint8_t smem_raw[];
@@ -97,13 +99,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int i0 = a.q_begin + tile * TQ;
   const int i_last = min(i0 + TQ, a.q_begin + a.q_len) - 1;
   const int nv_max = visible_kernels(i_last, 32, 16);
-  const int n_kt = (nv_max + 127) >> 7;
+  const int n_kt = (nv_max + 127) >> 7;  // pass-2 tiles (stage-1 kernels)
+  // pass-1 tiles: the same kernels, or the coarse kernels (128 tokens at stride
+  // 64) of the LSE approximation; the host sends only rows i >= 127 here
+  const int n_kt1 = a.approx ? (visible_kernels(i_last, 128, 64) + 127) >> 7 : n_kt;
 
   if (n_kt == 0) {  // no row of this tile sees a complete kernel
     if (a.score_lse && threadIdx.x < 128) {
       const int i = i0 + (int)threadIdx.x / G;
       if (i <= i_last)
-        a.score_lse[(size_t)(g * G + threadIdx.x % G) * a.q_len + (i - a.q_begin)] = -INFINITY;
+        a.score_lse[(size_t)(g * G + threadIdx.x % G) * a.o_len + (i - a.o_begin)] = -INFINITY;
     }
     return;
   }
@@ -131,25 +136,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const int total_it = 2 * n_kt;
+  const int total_it = n_kt1 + n_kt;
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
+      if (a.approx) tma_prefetch_desc(&tm_k2);
       mbar_expect_tx(S.q_full, kTileBytes);
       tma_load_3d(S.q, &tm_q, S.q_full, 0, g * G, i0);
       tma_load_3d(S.q + kTileBytes / 2, &tm_q, S.q_full, 64, g * G, i0);
       int issued = 0;
       for (int it = 0; it < total_it; ++it) {
         const int s = it % kStages;
-        const int jt = it < n_kt ? it : it - n_kt;
+        const int jt = it < n_kt1 ? it : it - n_kt1;
+        const CUtensorMap* tm = (it < n_kt1 && a.approx) ? &tm_k2 : &tm_k;
         if (!mbar_wait(S.kv_empty + 8 * s, ((it / kStages) & 1) ^ 1, a.wait)) break;
         const uint32_t dst = S.k + s * kTileBytes;
         mbar_expect_tx(S.kv_full + 8 * s, kTileBytes);
-        tma_load_3d(dst, &tm_k, S.kv_full + 8 * s, 0, g, jt * 128);
-        tma_load_3d(dst + kTileBytes / 2, &tm_k, S.kv_full + 8 * s, 64, g, jt * 128);
+        tma_load_3d(dst, tm, S.kv_full + 8 * s, 0, g, jt * 128);
+        tma_load_3d(dst + kTileBytes / 2, tm, S.kv_full + 8 * s, 64, g, jt * 128);
         issued = it + 1;
       }
       // never leave a copy in flight: wait (bounded) for the last loads to land
@@ -170,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(S.acc_empty + 8 * b, ((it >> 1) & 1) ^ 1, a.wait)) break;
         tc_fence_after();
         const uint32_t ks = S.k + s * kTileBytes;
-        const uint32_t a_base = it < n_kt ? S.q : ks;   // pass 1: rows = Q; pass 2: rows = K^C1
-        const uint32_t b_base = it < n_kt ? ks : S.q;
+        const uint32_t a_base = it < n_kt1 ? S.q : ks;  // pass 1: rows = Q; pass 2: rows = K^C1
+        const uint32_t b_base = it < n_kt1 ? ks : S.q;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
@@ -194,10 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + cg * kCols;
     const int tq_r = r / G;
     const int i_r = i0 + tq_r;
-    const int nv_r = i_r <= i_last ? visible_kernels(i_r, 32, 16) : 0;
+    // pass-1 kernel count of row r (coarse kernels in the approximation)
+    const int nv_r = i_r > i_last ? 0 : (a.approx ? visible_kernels(i_r, 128, 64)
+                                                  : visible_kernels(i_r, 32, 16));
     const float c = a.scale_log2;
     float vmax = -INFINITY, l = 0.f;
-    float* out_g = a.s_shared + (size_t)g * a.q_len * a.ld;
+    float* out_g = a.s_shared + (size_t)g * a.o_len * a.ld;
     // POOL: per token of this column group, the S^cmp row and the number of
     // blocks it holds (i/B; 0 for rows past the tile's end)
     float* cmp_row[TPG];
@@ -208,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < TPG; ++t) {
         const int i = i0 + cg * TPG + t;
         const bool in = i <= i_last;
-        cmp_row[t] = a.s_cmp + ((size_t)g * a.q_len + (in ? i - a.q_begin : 0)) * a.ld_cmp;
+        cmp_row[t] = a.s_cmp + ((size_t)g * a.o_len + (in ? i - a.o_begin : 0)) * a.ld_cmp;
         cmp_lim[t] = in ? (i >> 6) : 0;
       }
     }
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(S.acc_empty + 8 * b);  // TMEM buffer free again
-      if (it < n_kt) {
+      if (it < n_kt1) {
         // pass 1: row r, kernels it*128 + kCols*cg .. +31
         const int jb = it * 128 + cg * kCols;
         if (jb + 32 > nv_r) {
@@ -256,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l += (acc01.x + acc01.y) + (acc23.x + acc23.y);
         }
-        if (it == n_kt - 1) {
+        if (it == n_kt1 - 1) {
           // merge the column groups' statistics of row r
           s_part[(cg * 128 + r) * 2 + 0] = vmax;
           s_part[(cg * 128 + r) * 2 + 1] = l;
@@ -273,18 +282,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float mx = s_part[(x * 128 + r) * 2];
               if (mx != -INFINITY) L += s_part[(x * 128 + r) * 2 + 1] * fast_exp2((mx - M) * c);
             }
-            const float lse2 = L > 0.f ? M * c + __log2f(L) : -INFINITY;
+            // the approximation adds log2(s_C2 / s_C1) = 2: each coarse kernel
+            // stands for four stage-1 kernels
+            const float lse2 = L > 0.f ? M * c + __log2f(L) + (a.approx ? 2.0f : 0.0f) : -INFINITY;
             s_lse2[r] = -lse2;  // stored negated: pass 2 adds it
             if (a.score_lse && i_r <= i_last)
-              a.score_lse[(size_t)(g * G + r % G) * a.q_len + (i_r - a.q_begin)] = lse2 * kLn2;
+              a.score_lse[(size_t)(g * G + r % G) * a.o_len + (i_r - a.o_begin)] = lse2 * kLn2;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(S.lse_ready);
           if (!mbar_wait(S.lse_ready, 1, a.wait)) break;  // all 128 lse2 in smem
         }
       } else {
-        // pass 2: kernel j = (it - n_kt)*128 + r; this group's columns = tokens
-        const int jt = it - n_kt;
+        // pass 2: kernel j = (it - n_kt1)*128 + r; this group's columns = tokens
+        const int jt = it - n_kt1;
         const int j = jt * 128 + r;
         static_assert(G <= kCols, "a token's heads must fit in one column group");
         const float4* lse4 = reinterpret_cast<const float4*>(s_lse2 + cg * kCols);
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (POOL) {
             pv[t] = vis ? ssum : -INFINITY;
           } else {
-            if (vis) out_g[(size_t)(i - a.q_begin) * a.ld + j] = ssum;
+            if (vis) out_g[(size_t)(i - a.o_begin) * a.ld + j] = ssum;
           }
         }
         if constexpr (POOL) {
@@ -361,52 +372,91 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+struct ScoreLaunch {
+  const uint16_t *q, *kc1, *kc2;  // kc2: coarse kernels (approx only)
+  int n, h_q, h_kv;
+  int q_begin, q_len;             // rows to compute
+  int o_begin, o_len;             // row range of the output buffers
+  float scale;
+  float* out;                     // S^shared (or S^cmp when pooled)
+  int ld;
+  float* score_lse;
+  int approx;
+};
+
 template <int G, bool POOL>
-int launch_score_g(const uint16_t* q, const uint16_t* kc1, int n, int h_q, int h_kv, int q_begin,
-                   int q_len, float scale, float* s_out, int ld, float* score_lse,
-                   cudaStream_t st) {
+int launch_score_g(const ScoreLaunch& L, cudaStream_t st) {
   constexpr int TQ = 128 / G;
-  const int nc = n >= 32 ? (n - 32) / 16 + 1 : 0;
-  CUtensorMap tm_q, tm_k;
-  if (!make_tmap_3d(&tm_q, q, 128, h_q, n, 256, (uint64_t)h_q * 256, 64, G, TQ))
+  const int nc = L.n >= 32 ? (L.n - 32) / 16 + 1 : 0;
+  CUtensorMap tm_q, tm_k, tm_k2;
+  if (!make_tmap_3d(&tm_q, L.q, 128, L.h_q, L.n, 256, (uint64_t)L.h_q * 256, 64, G, TQ))
     return INFV2_ERR_CUDA;
   // K^C1 map; an empty K^C1 (nc == 0) still needs a valid map, one row is enough
-  if (!make_tmap_3d(&tm_k, kc1, 128, h_kv, nc > 0 ? nc : 1, 256, (uint64_t)h_kv * 256, 64, 1, 128))
+  if (!make_tmap_3d(&tm_k, L.kc1, 128, L.h_kv, nc > 0 ? nc : 1, 256, (uint64_t)L.h_kv * 256, 64, 1,
+                    128))
     return INFV2_ERR_CUDA;
+  if (L.approx) {
+    const int nc2 = num_coarse_kernels(L.n);
+    if (!make_tmap_3d(&tm_k2, L.kc2, 128, L.h_kv, nc2 > 0 ? nc2 : 1, 256, (uint64_t)L.h_kv * 256,
+                      64, 1, 128))
+      return INFV2_ERR_CUDA;
+  } else {
+    tm_k2 = tm_k;  // unused
+  }
   constexpr int TPG = kCols / G > 0 ? kCols / G : 1;
   const int smem = kTileBytes * (1 + kStages) + 128 * 4 + kColGroups * 128 * 2 * 4 +
                    (3 * kColGroups * 4 * TPG + 2) * 4 +
                    8 * (2 + 2 * kStages + 4 + kColGroups) + 16 + 1024;
   if (!set_smem(score_kernel<G, POOL>, smem)) return INFV2_ERR_CUDA;
   ScoreArgs a;
-  a.q_begin = q_begin;
-  a.q_len = q_len;
-  a.n_tiles = (q_len + TQ - 1) / TQ;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.ld = ld;
-  a.s_shared = POOL ? nullptr : s_out;
-  a.s_cmp = POOL ? s_out : nullptr;
-  a.ld_cmp = ld;
-  a.score_lse = score_lse;
+  a.q_begin = L.q_begin;
+  a.q_len = L.q_len;
+  a.n_tiles = (L.q_len + TQ - 1) / TQ;
+  a.o_begin = L.o_begin;
+  a.o_len = L.o_len;
+  a.approx = L.approx;
+  a.scale_log2 = L.scale * 1.4426950408889634f;
+  a.ld = L.ld;
+  a.s_shared = POOL ? nullptr : L.out;
+  a.s_cmp = POOL ? L.out : nullptr;
+  a.ld_cmp = L.ld;
+  a.score_lse = L.score_lse;
   a.wait = wait_ctx();
-  dim3 grid(a.n_tiles, h_kv);
-  score_kernel<G, POOL><<<grid, kThreads, smem, st>>>(tm_q, tm_k, a);
+  dim3 grid(a.n_tiles, L.h_kv);
+  score_kernel<G, POOL><<<grid, kThreads, smem, st>>>(tm_q, tm_k, tm_k2, a);
   return launch_status(cudaGetLastError());
 }
 
 template <bool POOL>
-int launch_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
-                  int q_begin, int q_len, float* out, int ld, float* score_lse, cudaStream_t st) {
-  if (q_len <= 0) return INFV2_OK;
-  const int G = p->h_q / p->h_kv;
-  switch (G) {
-    case 1: return launch_score_g<1, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
-    case 2: return launch_score_g<2, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
-    case 4: return launch_score_g<4, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
-    case 8: return launch_score_g<8, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
-    case 16: return launch_score_g<16, POOL>(q, kc1, n, p->h_q, p->h_kv, q_begin, q_len, p->scale, out, ld, score_lse, st);
+int launch_scores(const infv2_params* p, const ScoreLaunch& L, cudaStream_t st) {
+  if (L.q_len <= 0) return INFV2_OK;
+  switch (p->h_q / p->h_kv) {
+    case 1: return launch_score_g<1, POOL>(L, st);
+    case 2: return launch_score_g<2, POOL>(L, st);
+    case 4: return launch_score_g<4, POOL>(L, st);
+    case 8: return launch_score_g<8, POOL>(L, st);
+    case 16: return launch_score_g<16, POOL>(L, st);
     default: return INFV2_ERR_UNSUPPORTED;
   }
+}
+
+ScoreLaunch make_launch(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
+                        int q_begin, int q_len, float* out, int ld, float* score_lse) {
+  ScoreLaunch L;
+  L.q = q;
+  L.kc1 = kc1;
+  L.kc2 = nullptr;
+  L.n = n;
+  L.h_q = p->h_q;
+  L.h_kv = p->h_kv;
+  L.q_begin = L.o_begin = q_begin;
+  L.q_len = L.o_len = q_len;
+  L.scale = p->scale;
+  L.out = out;
+  L.ld = ld;
+  L.score_lse = score_lse;
+  L.approx = 0;
+  return L;
 }
 
 }  // namespace
@@ -414,13 +464,37 @@ int launch_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
 int launch_block_scores(const infv2_params* p, const uint16_t* q, const uint16_t* kc1, int n,
                         int q_begin, int q_len, float* s_shared, int ld, float* score_lse,
                         cudaStream_t st) {
-  return launch_scores<false>(p, q, kc1, n, q_begin, q_len, s_shared, ld, score_lse, st);
+  return launch_scores<false>(p, make_launch(p, q, kc1, n, q_begin, q_len, s_shared, ld, score_lse),
+                              st);
+}
+
+int launch_block_scores_approx(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
+                               const uint16_t* kc2, int n, int q_begin, int q_len,
+                               float* s_shared, int ld, float* score_lse, cudaStream_t st) {
+  // rows that see no coarse kernel (i < 4*l_c1 - 1 = 127) keep the exact LSE
+  constexpr int kFirstCoarse = 127;
+  const int end = q_begin + q_len;
+  ScoreLaunch L = make_launch(p, q, kc1, n, q_begin, q_len, s_shared, ld, score_lse);
+  if (q_begin < kFirstCoarse) {
+    L.q_len = (end < kFirstCoarse ? end : kFirstCoarse) - q_begin;
+    const int st1 = launch_scores<false>(p, L, st);
+    if (st1 != INFV2_OK) return st1;
+  }
+  if (end > kFirstCoarse) {
+    L.q_begin = q_begin > kFirstCoarse ? q_begin : kFirstCoarse;
+    L.q_len = end - L.q_begin;
+    L.kc2 = kc2;
+    L.approx = 1;
+    return launch_scores<false>(p, L, st);
+  }
+  return INFV2_OK;
 }
 
 int launch_block_scores_pooled(const infv2_params* p, const uint16_t* q, const uint16_t* kc1,
                                int n, int q_begin, int q_len, float* s_cmp, int ld_cmp,
                                cudaStream_t st) {
-  return launch_scores<true>(p, q, kc1, n, q_begin, q_len, s_cmp, ld_cmp, nullptr, st);
+  return launch_scores<true>(p, make_launch(p, q, kc1, n, q_begin, q_len, s_cmp, ld_cmp, nullptr),
+                             st);
 }
 
 }  // namespace infv2
@@ -460,4 +534,25 @@ extern "C" int infv2_block_scores_pooled(const infv2_params* p, const void* q, c
   return launch_block_scores_pooled(p, static_cast<const uint16_t*>(q),
                                     static_cast<const uint16_t*>(kc1), n, q_begin, q_len, s_cmp,
                                     ld_cmp, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int infv2_block_scores_approx(const infv2_params* p, const void* q, const void* kc1,
+                                         const void* kc2, int n, int q_begin, int q_len,
+                                         float* s_shared, int ld, float* score_lse,
+                                         infv2_stream_t stream) {
+  int st = infv2_check_params(p);
+  if (st != INFV2_OK) return st;
+  if (n < 0 || q_begin < 0 || q_len < 0 || q_begin + q_len > n) return INFV2_ERR_INVALID_ARG;
+  if (q_len == 0) return INFV2_OK;
+  if (!q || !s_shared) return INFV2_ERR_INVALID_ARG;
+  const int nc = infv2_num_kernels(p, n);
+  if (nc > 0 && !kc1) return INFV2_ERR_INVALID_ARG;
+  if (num_coarse_kernels(n) > 0 && q_begin + q_len > 127 && !kc2) return INFV2_ERR_INVALID_ARG;
+  if (ld < nc || ld % 4 != 0) return INFV2_ERR_INVALID_ARG;
+  if (nc == 0 && score_lse == nullptr) return INFV2_OK;
+  const void* kc1_map = kc1 ? kc1 : q;  // any valid address when no kernel exists
+  return launch_block_scores_approx(p, static_cast<const uint16_t*>(q),
+                                    static_cast<const uint16_t*>(kc1_map),
+                                    static_cast<const uint16_t*>(kc2), n, q_begin, q_len, s_shared,
+                                    ld, score_lse, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -23,6 +23,7 @@ SYMBOLS = [
     "infv2_sparse_attn", "infv2_dense_attn", "infv2_prefill_workspace_size", "infv2_prefill",
     "infv2_decode_workspace_size", "infv2_decode", "infv2_select_blocks_noalloc",
     "infv2_selftest_timeout", "infv2_block_scores_pooled", "infv2_select_topk_pooled",
+    "infv2_compress_k2", "infv2_block_scores_approx",
 ]
 
 
@@ -31,7 +32,7 @@ class Params(ctypes.Structure):
                 ("pool_l", ctypes.c_int), ("pool_s", ctypes.c_int), ("n_init", ctypes.c_int),
                 ("n_local", ctypes.c_int), ("k", ctypes.c_int), ("h_q", ctypes.c_int),
                 ("h_kv", ctypes.c_int), ("d", ctypes.c_int), ("scale", ctypes.c_float),
-                ("window", ctypes.c_int)]
+                ("window", ctypes.c_int), ("lse_approx", ctypes.c_int)]
 
 
 class Infv2Error(RuntimeError):
@@ -63,6 +64,8 @@ def lib():
         L.infv2_block_scores.argtypes = [P, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_block_scores_pooled.argtypes = [P, vp, vp, i, i, i, vp, i, vp]
+        L.infv2_compress_k2.argtypes = [P, vp, i, vp, vp]
+        L.infv2_block_scores_approx.argtypes = [P, vp, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk_pooled.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_sparse_attn.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
         L.infv2_dense_attn.argtypes = [P, vp, vp, vp, i, vp, vp, vp]
@@ -86,10 +89,10 @@ def _check(st: int, where: str):
 
 
 def params(h_q: int, h_kv: int, k: int = 64, n_init: int = 1, n_local: int = 2,
-           scale: float | None = None, window: int = 0) -> Params:
+           scale: float | None = None, window: int = 0, lse_approx: int = 0) -> Params:
     p = Params()
     lib().infv2_default_params(ctypes.byref(p), h_q, h_kv)
-    p.k, p.n_init, p.n_local, p.window = k, n_init, n_local, window
+    p.k, p.n_init, p.n_local, p.window, p.lse_approx = k, n_init, n_local, window, lse_approx
     if scale is not None:
         p.scale = scale
     return p
@@ -146,6 +149,33 @@ def infv2_compress_k(p: Params, k: torch.Tensor, kc1: torch.Tensor | None = None
     _check(lib().infv2_compress_k(ctypes.byref(p), _ptr(k), n, _ptr(kc1) if kc1.numel() else None,
                                   _stream(stream)), "infv2_compress_k")
     return kc1
+
+
+def num_coarse_kernels(p: Params, n: int) -> int:
+    """Coarse kernels of the LSE approximation (length 4*l_c1, stride 4*s_c1)."""
+    return (n - 4 * p.l_c1) // (4 * p.s_c1) + 1 if n >= 4 * p.l_c1 else 0
+
+
+def infv2_compress_k2(p: Params, k: torch.Tensor, kc2: torch.Tensor | None = None, stream=None):
+    n = k.shape[0]
+    if kc2 is None:
+        kc2 = torch.empty((num_coarse_kernels(p, n), p.h_kv, p.d), dtype=torch.bfloat16,
+                          device=k.device)
+    _check(lib().infv2_compress_k2(ctypes.byref(p), _ptr(k), n, _ptr(kc2) if kc2.numel() else None,
+                                   _stream(stream)), "infv2_compress_k2")
+    return kc2
+
+
+def infv2_block_scores_approx(p: Params, q, kc1, kc2, n: int, q_begin: int, q_len: int,
+                              s_shared=None, ld: int | None = None, score_lse=None, stream=None):
+    ld = shared_ld(n) if ld is None else ld
+    if s_shared is None:
+        s_shared = torch.zeros((p.h_kv, q_len, ld), dtype=torch.float32, device=q.device)
+    _check(lib().infv2_block_scores_approx(
+        ctypes.byref(p), _ptr(q), _ptr(kc1) if kc1.numel() else None,
+        _ptr(kc2) if kc2.numel() else None, n, q_begin, q_len, _ptr(s_shared), ld,
+        _ptr(score_lse), _stream(stream)), "infv2_block_scores_approx")
+    return s_shared
 
 
 def infv2_block_scores(p: Params, q, kc1, n: int, q_begin: int, q_len: int, s_shared=None,
