@@ -66,6 +66,7 @@ def _declare(L):
     L.orc_prefill_rows.argtypes = [P, vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp]
     L.orc_select_rows.argtypes = [P, vp, i, vp, i, vp, vp, i]
     L.orc_attend_rows.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
+    L.orc_attend_bwd_rows.argtypes = [P, vp, vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp]
     return L
 
 
@@ -260,3 +261,21 @@ def attend_rows(p: Params, q, k, v, rows, idx):
     _L().orc_attend_rows(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(rows), nr,
                           _ptr(idx), _ptr(o), _ptr(lse))
     return o, lse
+
+
+def attend_bwd_rows(p: Params, q, k, v, d_o, rows, idx, o):
+    """Backward of the attention at the given rows (see oracle.c).
+    o: [nrows, h_q, d] forward output (float); idx: [nrows, h_kv, k].
+    Returns dq [nrows, h_q, d] and dk, dv [n, h_kv, d] summed over those rows."""
+    q, k, v, d_o = (_c(x, np.uint16) for x in (q, k, v, d_o))
+    rows = _c(rows, np.int32)
+    idx = _c(idx, np.int32)
+    o = _c(np.asarray(o, np.float64), np.float64)
+    n = k.shape[0]
+    nr = len(rows)
+    dq = np.zeros((nr, p.h_q, p.d), np.float64)
+    dk = np.zeros((n, p.h_kv, p.d), np.float64)
+    dv = np.zeros((n, p.h_kv, p.d), np.float64)
+    _L().orc_attend_bwd_rows(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(d_o), n, _ptr(rows),
+                             nr, _ptr(idx), _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv

@@ -28,6 +28,10 @@
  *  - the local set is {b_i - n_local + 1 .. b_i} (own block included);
  *  - k counts every selected block, init and local included;
  *  - equal block scores are ordered by lower block index;
+ *  - backward (training; the arXiv summary's Appendix A returns the
+ *    log-sum-exp for it): the FlashAttention-style gradients of the attention
+ *    with the block lists fixed (selection is not differentiated); D = dO . O
+ *    uses the forward output O that the caller holds;
  *  - LSE approximation (optional): K^C2 is rounded to bf16 like K^C1, a coarse
  *    kernel is visible under the same rule, the estimate is the log-sum-exp
  *    over the visible coarse kernels plus log(s_C2 / s_C1) (each coarse kernel
@@ -410,6 +414,95 @@ void orc_select_rows(const orc_params* p, const double* shared, int ld, const in
 }
 
 /* Attention alone on given block lists idx [nrows][h_kv][k]. */
+/* Backward of orc_attend_row for query i and the heads of group g:
+ *   P_t  = softmax over the listed visible tokens t of scale * q_h . k_t
+ *   D_h  = dO_h . O_h          (O_h = o_in, the forward output)
+ *   dS_t = P_t * (dO_h . v_t - D_h)
+ *   dq_h = scale * sum_t dS_t k_t;  dk_t += scale * dS_t q_h;  dv_t += P_t dO_h
+ * o_in, dq_out: [G][d] fp64; d_o: bf16 [n, h_q, d]; dk_acc, dv_acc: fp64
+ * [n, h_kv, d], added to. */
+void orc_attend_bwd_row(const orc_params* p, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const uint16_t* d_o, int i, int g, const int* idx,
+                        int cnt, const double* o_in, double* dq_out, double* dk_acc,
+                        double* dv_acc) {
+    int G = p->h_q / p->h_kv;
+    int ntok = 0;
+    int* tok = (int*)malloc(sizeof(int) * ((size_t)cnt * p->B + 1));
+    for (int r = 0; r < cnt; ++r) {
+        if (idx[r] < 0) continue;
+        for (int t = idx[r] * p->B; t < (idx[r] + 1) * p->B && t <= i; ++t) tok[ntok++] = t;
+    }
+    double* P = (double*)malloc(sizeof(double) * (ntok + 1));
+    for (int hh = 0; hh < G; ++hh) {
+        int h = g * G + hh;
+        const uint16_t* qr = q + ((size_t)i * p->h_q + h) * p->d;
+        const uint16_t* dor = d_o + ((size_t)i * p->h_q + h) * p->d;
+        double* dq = dq_out + (size_t)hh * p->d;
+        for (int c = 0; c < p->d; ++c) dq[c] = 0.0;
+        if (ntok == 0) continue;
+        double m = -INFINITY;
+        for (int a = 0; a < ntok; ++a) {
+            const uint16_t* kr = k + ((size_t)tok[a] * p->h_kv + g) * p->d;
+            double dot = 0.0;
+            for (int c = 0; c < p->d; ++c) dot += bf16_value(qr[c]) * bf16_value(kr[c]);
+            P[a] = p->scale * dot;
+            if (P[a] > m) m = P[a];
+        }
+        double L = 0.0;
+        for (int a = 0; a < ntok; ++a) { P[a] = exp(P[a] - m); L += P[a]; }
+        for (int a = 0; a < ntok; ++a) P[a] /= L;
+        double D = 0.0;
+        for (int c = 0; c < p->d; ++c) D += bf16_value(dor[c]) * o_in[(size_t)hh * p->d + c];
+        for (int a = 0; a < ntok; ++a) {
+            size_t kv = ((size_t)tok[a] * p->h_kv + g) * p->d;
+            double dp = 0.0;
+            for (int c = 0; c < p->d; ++c) dp += bf16_value(dor[c]) * bf16_value(v[kv + c]);
+            double ds = P[a] * (dp - D);
+            for (int c = 0; c < p->d; ++c) {
+                dq[c] += p->scale * ds * bf16_value(k[kv + c]);
+                dk_acc[kv + c] += p->scale * ds * bf16_value(qr[c]);
+                dv_acc[kv + c] += P[a] * bf16_value(dor[c]);
+            }
+        }
+    }
+    free(P);
+    free(tok);
+}
+
+/* Backward over the given query rows of one n-token sequence.
+ *   o_in   [nrows][h_q][d] fp64: the forward output at those rows
+ *   idx    [nrows][h_kv][k]
+ *   dq_out [nrows][h_q][d]; dk_out, dv_out [n][h_kv][d] (overwritten: the
+ *   sums over the given rows only) */
+void orc_attend_bwd_rows(const orc_params* p, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const uint16_t* d_o, int n, const int* rows,
+                         int nrows, const int* idx, const double* o_in, double* dq_out,
+                         double* dk_out, double* dv_out) {
+    int G = p->h_q / p->h_kv;
+    size_t sz = (size_t)n * p->h_kv * p->d;
+    memset(dk_out, 0, sizeof(double) * sz);
+    memset(dv_out, 0, sizeof(double) * sz);
+#pragma omp parallel
+    {
+        double* dk = (double*)calloc(sz, sizeof(double));
+        double* dv = (double*)calloc(sz, sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r)
+            for (int g = 0; g < p->h_kv; ++g)
+                orc_attend_bwd_row(p, q, k, v, d_o, rows[r], g,
+                                   idx + ((size_t)r * p->h_kv + g) * p->k, p->k,
+                                   o_in + ((size_t)r * p->h_q + g * G) * p->d,
+                                   dq_out + ((size_t)r * p->h_q + g * G) * p->d, dk, dv);
+#pragma omp critical
+        for (size_t x = 0; x < sz; ++x) {
+            dk_out[x] += dk[x];
+            dv_out[x] += dv[x];
+        }
+        free(dk);
+        free(dv);
+    }
+}
+
 void orc_attend_rows(const orc_params* p, const uint16_t* q, const uint16_t* k,
                      const uint16_t* v, const int* rows, int nrows, const int* idx,
                      double* o_out, double* lse_out) {

@@ -472,4 +472,60 @@ def pin_early_rows_are_dense():
         assert np.allclose(out["o"][r], o, rtol=1e-12, atol=1e-12), i
 
 
+# --------------------------------------------------------------------------
+# backward of the attention (block lists fixed)
+# --------------------------------------------------------------------------
+
+def _bwd_problem(n=300, h_q=4, h_kv=2, d=16, seed=31, k=3):
+    sh, data = _small_problem(n=n, h_q=h_q, h_kv=h_kv, d=d, seed=seed, k=k)
+    p = oracle.params(sh)
+    rows = np.arange(n, dtype=np.int32)
+    fwd = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows)
+    rng = np.random.default_rng(seed + 1)
+    d_o = _bf16(rng.standard_normal((n, h_q, d)))
+    return sh, p, data, rows, fwd, d_o
+
+
+def pin_attend_bwd_matches_autograd():
+    """Every row's block-sparse causal attention written as one masked softmax
+    in torch fp64; autograd of sum(O * dO) gives dq, dk, dv."""
+    sh, p, data, rows, fwd, d_o = _bwd_problem()
+    n, G = sh.n, sh.G
+    dq, dk, dv = oracle.attend_bwd_rows(p, data["q"], data["k"], data["v"], d_o, rows, fwd["idx"], fwd["o"])
+    q, k, v, go = (torch.from_numpy(_f64(x)).requires_grad_(True) for x in (data["q"], data["k"], data["v"], d_o))
+    t = torch.arange(n)
+    mask = torch.zeros((sh.h_kv, n, n), dtype=torch.bool)
+    for i in range(n):
+        for g in range(sh.h_kv):
+            blocks = torch.tensor([b for b in fwd["idx"][i, g] if b >= 0])
+            mask[g, i] = (t <= i) & torch.isin(t // 64, blocks)
+    kk = k.repeat_interleave(G, dim=1).permute(1, 0, 2)      # [h_q, n, d]
+    vv = v.repeat_interleave(G, dim=1).permute(1, 0, 2)
+    qq = q.permute(1, 0, 2)
+    z = qq @ kk.transpose(1, 2) / np.sqrt(sh.d)
+    z = z.masked_fill(~mask.repeat_interleave(G, dim=0), -np.inf)
+    o = torch.softmax(z, dim=-1) @ vv                        # [h_q, n, d]
+    (o * go.detach().permute(1, 0, 2)).sum().backward()
+    assert np.allclose(o.detach().permute(1, 0, 2).numpy(), fwd["o"], rtol=0, atol=1e-12)
+    assert np.allclose(dq, q.grad.numpy(), rtol=0, atol=1e-11), np.abs(dq - q.grad.numpy()).max()
+    assert np.allclose(dk, k.grad.numpy(), rtol=0, atol=1e-11), np.abs(dk - k.grad.numpy()).max()
+    assert np.allclose(dv, v.grad.numpy(), rtol=0, atol=1e-11), np.abs(dv - v.grad.numpy()).max()
+
+
+def pin_attend_bwd_closed_forms():
+    """Row 0 sees token 0 only: P = 1, so dq_0 = 0 and token 0 receives dv = dO_0
+    (plus the later rows' shares).  Over all rows, sum_t dv_t = sum of dO over
+    the rows and the group's heads, and sum_t dk_t = 0 (sum_t dS_t = 0)."""
+    sh, p, data, rows, fwd, d_o = _bwd_problem(n=260, seed=41)
+    dq, dk, dv = oracle.attend_bwd_rows(p, data["q"], data["k"], data["v"], d_o, rows[:1],
+                                        fwd["idx"][:1], fwd["o"][:1])
+    assert np.all(dq[0] == 0.0)
+    assert np.allclose(dv[0], _f64(d_o)[0].reshape(sh.h_kv, sh.G, sh.d).sum(axis=1), rtol=0, atol=1e-14)
+    assert np.all(dk == 0.0) and np.all(dv[1:] == 0.0)
+    dq, dk, dv = oracle.attend_bwd_rows(p, data["q"], data["k"], data["v"], d_o, rows, fwd["idx"], fwd["o"])
+    go = _f64(d_o).reshape(sh.n, sh.h_kv, sh.G, sh.d).sum(axis=2)      # [n, h_kv, d]
+    assert np.allclose(dv.sum(axis=0), go.sum(axis=0), rtol=0, atol=1e-10)
+    assert np.allclose(dk.sum(axis=0), 0.0, rtol=0, atol=1e-10), np.abs(dk.sum(axis=0)).max()
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

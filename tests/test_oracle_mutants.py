@@ -29,6 +29,9 @@ MUTANTS = {
     "values_from_keys": ("const uint16_t* vr = v +", "const uint16_t* vr = k +"),
     "mean_divides_by_stride": ("orc_bf16_round(s / p->l_c1)", "orc_bf16_round(s / p->s_c1)"),
     "ties_away_from_zero": ("else if (rem == 0.5 && fmod(lo, 2.0) != 0.0) r = lo + 1.0;", "else if (rem == 0.5) r = lo + 1.0;"),
+    "bwd_drops_D": ("double ds = P[a] * (dp - D);", "double ds = P[a] * dp;"),
+    "bwd_dk_unscaled": ("dk_acc[kv + c] += p->scale * ds * bf16_value(qr[c]);", "dk_acc[kv + c] += ds * bf16_value(qr[c]);"),
+    "bwd_dv_from_ds": ("dv_acc[kv + c] += P[a] * bf16_value(dor[c]);", "dv_acc[kv + c] += ds * bf16_value(dor[c]);"),
     "kernel_window_short": ("t < j * p->s_c1 + p->l_c1; ++t", "t < j * p->s_c1 + p->l_c1 - 1; ++t"),
 }
 
