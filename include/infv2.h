@@ -195,6 +195,30 @@ int infv2_select_topk_pooled(const infv2_params* p, const float* s_cmp, int ld_c
 int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const void* v,
                       const int* idx, int n, void* o, float* lse, infv2_stream_t stream);
 
+/* Workspace bytes that infv2_sparse_attn_bwd needs for an n-token sequence
+ * (either mode: block lists or dense). */
+int infv2_sparse_attn_bwd_workspace_size(const infv2_params* p, int n, size_t* bytes);
+
+/* Backward of infv2_sparse_attn (or of the dense attention when idx is NULL)
+ * for training (arXiv summary, Appendix A: the forward's log-sum-exp is kept
+ * for the backward).  The block lists are fixed: the selection is not
+ * differentiated.  For every query i, head h of group g and visible token t of
+ * i's blocks, with P_t = exp(scale q_ih . k_t - lse[h, i]):
+ *   D_ih = dO_ih . O_ih   (O = the forward output passed in)
+ *   dS_t = P_t (dO_ih . v_t - D_ih)
+ *   dq_ih = scale sum_t dS_t k_t;  dk_t += scale dS_t q_ih;  dv_t += P_t dO_ih
+ *   q bf16 [n, h_q, d]; k, v bf16 [n, h_kv, d]; idx int32 [h_kv, n, k] or NULL
+ *   o bf16 [n, h_q, d] and lse fp32 [h_q, n] (natural) from the forward
+ *   d_o bf16 [n, h_q, d]
+ *   dq fp32 [n, h_q, d]; dk, dv fp32 [n, h_kv, d] (outputs, overwritten)
+ *   workspace: >= infv2_sparse_attn_bwd_workspace_size bytes, 256-byte aligned.
+ * dk and dv are sums over many queries added in an order that varies from run
+ * to run: equal inputs give results equal up to fp32 rounding. */
+int infv2_sparse_attn_bwd(const infv2_params* p, const void* q, const void* k, const void* v,
+                          const int* idx, int n, const void* o, const float* lse,
+                          const void* d_o, float* dq, float* dk, float* dv, void* workspace,
+                          size_t ws_bytes, infv2_stream_t stream);
+
 /* Dense causal attention with the same weights (MiniCPM4 blog: sequences of
  * at most k blocks switch to dense attention).  Layouts as infv2_sparse_attn. */
 int infv2_dense_attn(const infv2_params* p, const void* q, const void* k, const void* v, int n,

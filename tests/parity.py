@@ -59,3 +59,23 @@ def assert_outputs_close(o_gpu, o_orc, what=""):
     mx, mean = compare_outputs(o_gpu, o_orc)
     assert mx <= O_MAX_ABS and mean <= O_MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
     return mx, mean
+
+
+def assert_grads_close(got, want, name, rel_fro=5e-3, rel_max=1e-2):
+    """fp32 gradients against the fp64 oracle: relative Frobenius error of the
+    whole tensor and the largest element error relative to the largest
+    reference magnitude.  The GPU rounds P and dS to bf16 for its MMAs
+    (relative 2^-9 per element, averaging out over the sums)."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (name, got.shape, want.shape)
+    assert np.all(np.isfinite(got)), name
+    if np.abs(want).max() < 1e-9:
+        # an exactly-zero gradient (e.g. a query that sees one token): fp32
+        # rounding of dO.v - D leaves residues far below the data's scale
+        assert np.abs(got).max() < 1e-4, (name, np.abs(got).max())
+        return
+    scale = np.abs(want).max()
+    fro = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    mx = np.abs(got - want).max() / scale
+    assert fro <= rel_fro and mx <= rel_max, (name, fro, mx)

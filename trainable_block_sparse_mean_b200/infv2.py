@@ -23,7 +23,8 @@ SYMBOLS = [
     "infv2_sparse_attn", "infv2_dense_attn", "infv2_prefill_workspace_size", "infv2_prefill",
     "infv2_decode_workspace_size", "infv2_decode", "infv2_select_blocks_noalloc",
     "infv2_selftest_timeout", "infv2_block_scores_pooled", "infv2_select_topk_pooled",
-    "infv2_compress_k2", "infv2_block_scores_approx",
+    "infv2_compress_k2", "infv2_block_scores_approx", "infv2_sparse_attn_bwd_workspace_size",
+    "infv2_sparse_attn_bwd",
 ]
 
 
@@ -65,6 +66,8 @@ def lib():
         L.infv2_select_topk.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_block_scores_pooled.argtypes = [P, vp, vp, i, i, i, vp, i, vp]
         L.infv2_compress_k2.argtypes = [P, vp, i, vp, vp]
+        L.infv2_sparse_attn_bwd_workspace_size.argtypes = [P, i, ctypes.POINTER(sz)]
+        L.infv2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.infv2_block_scores_approx.argtypes = [P, vp, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk_pooled.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_sparse_attn.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
@@ -232,6 +235,29 @@ def infv2_sparse_attn(p: Params, q, k, v, idx, o=None, lse=None, stream=None):
     _check(lib().infv2_sparse_attn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), n,
                                    _ptr(o), _ptr(lse), _stream(stream)), "infv2_sparse_attn")
     return o
+
+
+def infv2_sparse_attn_bwd_workspace_size(p: Params, n: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().infv2_sparse_attn_bwd_workspace_size(ctypes.byref(p), n, ctypes.byref(out)),
+           "infv2_sparse_attn_bwd_workspace_size")
+    return out.value
+
+
+def infv2_sparse_attn_bwd(p: Params, q, k, v, idx, o, lse, d_o, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) in fp32 of the attention over idx (None: dense)."""
+    n = q.shape[0]
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    need = infv2_sparse_attn_bwd_workspace_size(p, n)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().infv2_sparse_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), n,
+                                       _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "infv2_sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def infv2_dense_attn(p: Params, q, k, v, o=None, lse=None, stream=None):
