@@ -251,6 +251,7 @@ def run_ours(args, rank, world, local_rank, dist):
     stage = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, chunk_rows)
     fused = _fused_pool_timing(args, infv2, torch, p, shape, q, k, ws, stream, chunk_rows, stage)
     approx = _lse_approx_timing(args, infv2, torch, shape, q, k, v, o, lse, stream, ms)
+    bwd = _backward_timing(args, infv2, torch, p, shape, q, k, v, ws, stream)
     # ---- end to end through host buffers
     e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_ranks)
     # ---- decode
@@ -306,6 +307,7 @@ def run_ours(args, rank, world, local_rank, dist):
         "stages": stage["per_kernel"],
         "fused_pool": fused,
         "lse_approx": approx,
+        "backward": bwd,
         "roofline": roof,
         "e2e": e2e,
         "decode": dec,
@@ -462,6 +464,41 @@ def _lse_approx_timing(args, infv2, torch, shape, q, k, v, o, lse, stream, exact
             "used_in_step": False,
             "note": "pass-1 log-sum-exp from the coarse kernels K^C2 (l=128, s=64); selection "
                     "differs from the exact path where the estimate reorders near-equal blocks"}
+
+
+def _backward_timing(args, infv2, torch, p, shape, q, k, v, ws, stream):
+    """The attention backward (dq, dk, dv) on the prefill's own block lists,
+    timed on the device; reported beside the forward step."""
+    n = shape.n
+    cu = [0, n]
+    idx = torch.empty((p.h_kv, n, p.k), dtype=torch.int32, device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((p.h_q, n), device=q.device)
+    infv2.infv2_prefill(p, q, k, v, cu, workspace=ws, idx_out=idx, o=o, lse=lse)
+    gen = torch.Generator(device=q.device)
+    gen.manual_seed(1)
+    d_o = torch.randn(q.shape, generator=gen, device=q.device).to(torch.bfloat16)
+    bws = torch.empty(infv2.infv2_sparse_attn_bwd_workspace_size(p, n), dtype=torch.uint8,
+                      device=q.device)
+
+    def step():
+        return infv2.infv2_sparse_attn_bwd(p, q, k, v, idx, o, lse, d_o, workspace=bws)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    attn = prefill_work(shape, n)["attn"]          # 4*d FLOP per (head, selected visible key)
+    executed = attn * 14.0 / 4.0                   # S, dP, dS.K (dq) + S, dP, P^T.dO, dS^T.Q (dk, dv)
+    return {"ms_per_step": round(ms, 3), "tflop_executed": round(executed / 1e12, 3),
+            "tflops_executed": round(executed / (ms / 1e3) / 1e12, 1),
+            "note": "dq, dk, dv in fp32 over the prefill's block lists (selection fixed)"}
 
 
 def _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks):
