@@ -220,6 +220,10 @@ def run_ours(args, rank, world, local_rank, dist):
     def step():
         infv2.infv2_prefill(p, q, k, v, cu, workspace=ws, o=o, lse=lse)
 
+    if args.only == "backward":  # profiling runs: the attention backward only
+        return {"metric": METRIC, "workload": args.workload,
+                "backward": _backward_timing(args, infv2, torch, p, shape, q, k, v, ws,
+                                             torch.cuda.current_stream())}
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -703,8 +707,8 @@ def main():
                     help="prefill workload: c3 (131072 tokens, the reported one) or c2 (32768)")
     ap.add_argument("--decode-small", action="store_true",
                     help="with --only decode: 8 sequences of 16k-32k tokens (profiler runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="prefill / decode: time only that part (for profiler runs)")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
+                    help="prefill / decode / backward: time only that part (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
