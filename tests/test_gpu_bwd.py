@@ -104,3 +104,37 @@ def test_bwd_workspace_too_small_is_rejected():
     with pytest.raises(infv2.Infv2Error) as e:
         infv2.infv2_sparse_attn_bwd(p, q, k, k, None, q, lse, q, workspace=ws)
     assert e.value.status == infv2.ERR_WORKSPACE
+
+
+@pytest.mark.slow
+def test_bwd_c2_full_size_sampled():
+    """The 32k workload through the prefill's own block lists: dq on sampled rows
+    against the oracle; dk, dv through invariants that hold at any size
+    (sum_t dv_t = sum of dO over the group's heads; sum_t dk_t = scale * sum_i
+    (sum_t dS_t) q_i, which is 0 up to D's use of the bf16 forward output)."""
+    sh = synth.CONFIGS["c2"]["shape"]
+    d = synth.make_prefill(sh, seed=0)
+    p, op = infv2.params_of(sh), oracle.params(sh)
+    n = sh.n
+    q, k, v = to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"])
+    idx = torch.empty((sh.h_kv, n, sh.k), dtype=torch.int32, device="cuda")
+    lse = torch.empty((sh.h_q, n), device="cuda")
+    o = infv2.infv2_prefill(p, q, k, v, [0, n], idx_out=idx, lse=lse)
+    d_o = synth.bf16_bits(np.random.default_rng(8).standard_normal((n, sh.h_q, sh.d)).astype(np.float32))
+    dq, dk, dv = infv2.infv2_sparse_attn_bwd(p, q, k, v, idx, o, lse, to_dev(d_o))
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    rows = np.unique(np.concatenate([[0, 63, 64, 4095, 4096, n - 1],
+                                     np.random.default_rng(1).integers(0, n, 60)])).astype(np.int32)
+    o_host = synth.bf16_to_f32(to_host_bits(o))[rows].astype(np.float64)
+    idx_rows = idx.cpu().numpy()[:, rows].transpose(1, 0, 2).copy()
+    rq, _, _ = oracle.attend_bwd_rows(op, d["q"], d["k"], d["v"], d_o, rows, idx_rows, o_host)
+    parity.assert_grads_close(dq.cpu().numpy()[rows], rq, "dq sampled")
+    go = synth.bf16_to_f32(d_o).astype(np.float64).reshape(n, sh.h_kv, sh.G, sh.d).sum(axis=2)
+    dvs = dv.cpu().numpy().astype(np.float64).sum(axis=0)
+    want = go.sum(axis=0)
+    # the GPU rounds P to bf16 for P^T dO: per (row, head) the weights sum to 1
+    # within ~2^-9 sqrt(sum P^2), a random error that grows as sqrt(rows * heads)
+    assert np.abs(dvs - want).max() <= 5e-3 * np.abs(want).max() + 0.5, np.abs(dvs - want).max()
+    dks = np.abs(dk.cpu().numpy().astype(np.float64).sum(axis=0)).max()
+    assert dks <= 2e-2 * np.abs(dk.cpu().numpy()).sum(axis=0).max(), dks

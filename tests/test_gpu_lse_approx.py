@@ -94,3 +94,13 @@ def test_decode_rejects_the_approximation():
     import ctypes
     size = ctypes.c_size_t()
     assert infv2.lib().infv2_decode_workspace_size(ctypes.byref(p), 4, 4096, ctypes.byref(size)) == infv2.ERR_UNSUPPORTED
+
+
+@pytest.mark.slow
+def test_prefill_approx_c3_sampled():
+    """The 128k workload with the approximation: sampled rows against the
+    oracle in the same mode."""
+    sh = synth.CONFIGS["c3"]["shape"]
+    data = synth.make_prefill(sh, seed=0)
+    dev = run_prefill(sh, data, [0, sh.n], lse_approx=1)
+    check_sequence(sh, data, dev, 0, sh.n, _rows(sh.n, 200, 3), dense=False, lse_approx=1)
