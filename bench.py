@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 from trainable_block_sparse_mean_b200 import synth  # noqa: E402
 
 METRIC = "sparse prefill tokens/s + TFLOP/s at 128k (% of peak); decode µs/token"
-WORKLOAD = "c3: prefill, single sequence n=131072, h_q=32, h_kv=2, d=128, bf16, top-k 64 blocks of 64, 128 needles"
+WORKLOAD = "prefill_128k: prefill, single sequence n=131072, h_q=32, h_kv=2, d=128, bf16, top-k 64 blocks of 64, 128 needles"
 B, D = 64, 128
 
 
@@ -579,7 +579,7 @@ def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, Decod
     split-KV attention, combine: 7 launches) is captured once into a CUDA graph,
     as a serving loop would run it, and the graphs are replayed in order (each
     replay appends its own token and advances seqlens on the device)."""
-    cfg = dict(synth.CONFIGS["c4"])
+    cfg = dict(synth.CONFIGS["decode_batch32"])
     if args.decode_small:   # profiler runs: 8 sequences of at most 32k tokens
         cfg.update(batch=8, len_lo=16384, len_hi=32768)
     sh = cfg["shape"]
@@ -619,7 +619,7 @@ def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, Decod
     peaks = measured_peaks()
     gbs = byts / (us / 1e6) / 1e9
     del graphs
-    return {"workload": "c4: batch 32, one query token each, cache lengths U[16384, 131072] "
+    return {"workload": "decode_batch32: batch 32, one query token each, cache lengths U[16384, 131072] "
                         "(seed-0 mean %.0f), h_q=32, h_kv=2, top-k 64" % data["lens"].mean(),
             "us_per_step": round(us, 2), "us_per_token_per_sequence": round(us, 2),
             "us_per_token_aggregate": round(us / cfg["batch"], 3),
@@ -635,7 +635,7 @@ def oracle_sample(target_s=12.0, seed=0):
     """Time the fp64 oracle on a bounded random sample of query rows of the
     128k workload (rows drawn uniformly; cost grows with the row index)."""
     import oracle
-    shape = synth.CONFIGS["c3"]["shape"]
+    shape = synth.CONFIGS["prefill_128k"]["shape"]
     data = synth.make_prefill(shape, seed=0)
     op = oracle.params(shape)
     rng = np.random.default_rng(seed)
@@ -659,7 +659,7 @@ def oracle_sample(target_s=12.0, seed=0):
 def run_reference(args):
     import oracle
     oracle.build()
-    shape = synth.CONFIGS["c3"]["shape"]
+    shape = synth.CONFIGS["prefill_128k"]["shape"]
     data = synth.make_prefill(shape, seed=0)
     op = oracle.params(shape)
     threads = oracle.num_threads()
@@ -703,8 +703,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["c3", "c2"], default="c3",
-                    help="prefill workload: c3 (131072 tokens, the reported one) or c2 (32768)")
+    ap.add_argument("--workload", choices=["prefill_128k", "prefill_32k"], default="prefill_128k",
+                    help="prefill workload: prefill_128k (131072 tokens, the reported one) or prefill_32k (32768)")
     ap.add_argument("--decode-small", action="store_true",
                     help="with --only decode: 8 sequences of 16k-32k tokens (profiler runs)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",

@@ -375,7 +375,7 @@ def pin_select_bruteforce():
 
 
 def pin_select_invariants():
-    sh = synth.CONFIGS["c1"]["shape"]
+    sh = synth.CONFIGS["prefill_2k"]["shape"]
     data = synth.make_prefill(sh, seed=0)
     p = oracle.params(sh)
     rows = np.array([0, 30, 31, 63, 64, 200, 511, 512, 513, 777, 1500, 2047])

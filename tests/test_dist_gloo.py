@@ -58,7 +58,7 @@ def test_reference_arm_non_zero_rank_exits_quietly():
 
 
 def test_prefill_work_matches_closed_form():
-    sh = synth.CONFIGS["c3"]["shape"]
+    sh = synth.CONFIGS["prefill_128k"]["shape"]
     w = bench.prefill_work(sh, sh.n)
     # two passes x 2*d FLOP per (head, query, visible kernel):
     # sum_i nv(i) with nv(i) = (i-31)//16 + 1 for i >= 31
@@ -74,7 +74,7 @@ def test_prefill_work_matches_closed_form():
 
 
 def test_decode_bytes_at_seed0_lengths():
-    cfg = synth.CONFIGS["c4"]
+    cfg = synth.CONFIGS["decode_batch32"]
     lens = synth.decode_lengths(cfg["batch"], cfg["len_lo"], cfg["len_hi"], 0)
     b = bench.decode_bytes(cfg["shape"], lens)
     assert 2.0e8 < b < 2.3e8          # ~213 MB: K^C1 rows + 4096 selected keys of K and V

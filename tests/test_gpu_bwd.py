@@ -107,12 +107,12 @@ def test_bwd_workspace_too_small_is_rejected():
 
 
 @pytest.mark.slow
-def test_bwd_c2_full_size_sampled():
+def test_bwd_32k_sampled():
     """The 32k workload through the prefill's own block lists: dq on sampled rows
     against the oracle; dk, dv through invariants that hold at any size
     (sum_t dv_t = sum of dO over the group's heads; sum_t dk_t = scale * sum_i
     (sum_t dS_t) q_i, which is 0 up to D's use of the bf16 forward output)."""
-    sh = synth.CONFIGS["c2"]["shape"]
+    sh = synth.CONFIGS["prefill_32k"]["shape"]
     d = synth.make_prefill(sh, seed=0)
     p, op = infv2.params_of(sh), oracle.params(sh)
     n = sh.n

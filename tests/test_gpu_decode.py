@@ -107,8 +107,8 @@ def _with_lengths(sh, lens, steps, cap, seed):
 
 
 @pytest.mark.slow
-def test_c4_full_size_sampled():
-    cfg = synth.CONFIGS["c4"]
+def test_decode_batch32_sampled():
+    cfg = synth.CONFIGS["decode_batch32"]
     sh = cfg["shape"]
     sample = [0, 7, 19, 31]
     data = synth.make_decode(sh, cfg["batch"], cfg["len_lo"], cfg["len_hi"], 3, seed=0, only=sample)

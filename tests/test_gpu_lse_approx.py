@@ -97,10 +97,10 @@ def test_decode_rejects_the_approximation():
 
 
 @pytest.mark.slow
-def test_prefill_approx_c3_sampled():
+def test_prefill_approx_128k_sampled():
     """The 128k workload with the approximation: sampled rows against the
     oracle in the same mode."""
-    sh = synth.CONFIGS["c3"]["shape"]
+    sh = synth.CONFIGS["prefill_128k"]["shape"]
     data = synth.make_prefill(sh, seed=0)
     dev = run_prefill(sh, data, [0, sh.n], lse_approx=1)
     check_sequence(sh, data, dev, 0, sh.n, _rows(sh.n, 200, 3), dense=False, lse_approx=1)

@@ -73,8 +73,8 @@ def _rows(n, count, seed):
     return np.unique(r).astype(np.int32)
 
 
-def test_c1_every_row():
-    sh = synth.CONFIGS["c1"]["shape"]
+def test_prefill_2k_every_row():
+    sh = synth.CONFIGS["prefill_2k"]["shape"]
     data = synth.make_prefill(sh, seed=0)
     dev = run_prefill(sh, data, [0, sh.n])
     st = check_sequence(sh, data, dev, 0, sh.n, np.arange(sh.n, dtype=np.int32), dense=False)
@@ -90,8 +90,8 @@ def test_medium_sizes(n, h_q, h_kv, k):
 
 
 @pytest.mark.slow
-def test_c2_full_size_sampled():
-    sh = synth.CONFIGS["c2"]["shape"]
+def test_prefill_32k_sampled():
+    sh = synth.CONFIGS["prefill_32k"]["shape"]
     data = synth.make_prefill(sh, seed=0)
     dev = run_prefill(sh, data, [0, sh.n])
     rows = _rows(sh.n, 120, 2)
@@ -100,8 +100,8 @@ def test_c2_full_size_sampled():
 
 
 @pytest.mark.slow
-def test_c3_full_size_sampled():
-    sh = synth.CONFIGS["c3"]["shape"]
+def test_prefill_128k_sampled():
+    sh = synth.CONFIGS["prefill_128k"]["shape"]
     data = synth.make_prefill(sh, seed=0)
     dev = run_prefill(sh, data, [0, sh.n])
     rows = _rows(sh.n, 48, 3)
@@ -121,8 +121,8 @@ def test_c3_full_size_sampled():
 
 
 @pytest.mark.slow
-def test_c5_varlen_switch_sweep():
-    cfg = synth.CONFIGS["c5"]
+def test_varlen_switch_sweep():
+    cfg = synth.CONFIGS["varlen_sweep"]
     sh = cfg["shape"]
     lengths = cfg["lengths"]
     data = synth.make_varlen(sh, lengths, seed=0)

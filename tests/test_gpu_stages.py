@@ -67,7 +67,7 @@ SCORE_REL = 2e-5   # fp32 tensor-core dot products + fp32 softmax vs fp64
 
 
 @pytest.mark.parametrize("n,h_q,h_kv,q_begin,q_len", [
-    (2048, 4, 1, 0, 2048),        # c1 shape, G=4 (32 tokens per tile)
+    (2048, 4, 1, 0, 2048),        # the 2k workload's shape, G=4 (32 tokens per tile)
     (3000, 32, 2, 0, 3000),       # G=16, ragged tail, 188 kernels (2 tiles)
     (3000, 32, 2, 1000, 1333),    # a chunk in the middle of the sequence
     (700, 8, 1, 0, 700),          # G=8

@@ -58,16 +58,16 @@ class Shape:
 # hyper-parameters: block 64, kernel 32, stride 16, pooling 5/4).
 CONFIGS = {
     # single 2k sequence, G=4, 8 blocks total: small enough for the oracle
-    "c1": dict(shape=Shape(n=2048, h_q=4, h_kv=1, k=8)),
+    "prefill_2k": dict(shape=Shape(n=2048, h_q=4, h_kv=1, k=8)),
     # single 32k sequence, G=16, 64 blocks (4096 keys), 32 needles
-    "c2": dict(shape=Shape(n=32768, h_q=32, h_kv=2, k=64, n_needles=32)),
+    "prefill_32k": dict(shape=Shape(n=32768, h_q=32, h_kv=2, k=64, n_needles=32)),
     # single 128k sequence, G=16, 64 blocks, 128 needles
-    "c3": dict(shape=Shape(n=131072, h_q=32, h_kv=2, k=64, n_needles=128)),
+    "prefill_128k": dict(shape=Shape(n=131072, h_q=32, h_kv=2, k=64, n_needles=128)),
     # batched decode: 32 sequences with cache lengths U[16384, 131072]
-    "c4": dict(shape=Shape(n=0, h_q=32, h_kv=2, k=64), batch=32,
+    "decode_batch32": dict(shape=Shape(n=0, h_q=32, h_kv=2, k=64), batch=32,
                len_lo=16384, len_hi=131072, steps=64),
     # dense/sparse switch sweep: eight sequences of 1k..96k tokens
-    "c5": dict(shape=Shape(n=0, h_q=32, h_kv=2, k=64),
+    "varlen_sweep": dict(shape=Shape(n=0, h_q=32, h_kv=2, k=64),
                lengths=(1024, 2048, 4096, 8192, 16384, 32768, 65536, 98304)),
 }
 
