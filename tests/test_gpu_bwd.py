@@ -56,7 +56,8 @@ def _run(sh, d, idx_np, seed):
     return (dq.cpu().numpy(), dk.cpu().numpy(), dv.cpu().numpy()), (rq, rk, rv)
 
 
-@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (3001, 32, 2, 16), (1500, 16, 2, 4)])
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (3001, 32, 2, 16), (1500, 16, 2, 4),
+                                         (1300, 2, 2, 6), (1100, 4, 2, 5)])
 def test_bwd_on_oracle_indices(n, h_q, h_kv, k):
     sh = synth.Shape(n=n, h_q=h_q, h_kv=h_kv, k=k)
     d = synth.make_prefill(sh, seed=n)

@@ -80,12 +80,14 @@ def run_and_check(shape, data, steps, check_seqs, check_steps):
     return stats
 
 
-def test_decode_small_mixed_lengths():
-    # dense (L+1 <= k*B) and sparse sequences, kernels completing during the run
-    sh = synth.Shape(n=0, h_q=16, h_kv=2, k=8)
+@pytest.mark.parametrize("h_q,h_kv,steps", [(16, 2, 40), (2, 2, 12), (4, 2, 12), (4, 1, 12)])
+def test_decode_small_mixed_lengths(h_q, h_kv, steps):
+    # dense (L+1 <= k*B) and sparse sequences, kernels completing during the run;
+    # group sizes 8, 1, 2 and 4
+    sh = synth.Shape(n=0, h_q=h_q, h_kv=h_kv, k=8)
     lens = np.array([0, 20, 31, 100, 511, 700, 3000, 5000], np.int32)
-    data = _with_lengths(sh, lens, steps=40, cap=5100, seed=3)
-    run_and_check(sh, data, 40, range(len(lens)), check_steps=set(range(40)))
+    data = _with_lengths(sh, lens, steps=steps, cap=5100, seed=3)
+    run_and_check(sh, data, steps, range(len(lens)), check_steps=set(range(steps)))
 
 
 def _with_lengths(sh, lens, steps, cap, seed):
