@@ -168,6 +168,16 @@ def measured_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def workload_config(shape, world):
+    """The `config` object of both arms' JSON lines (the same workload)."""
+    return {"workload": WORKLOAD, "n": shape.n, "h_q": shape.h_q, "h_kv": shape.h_kv,
+            "d": shape.d, "block": shape.B, "top_k_blocks": shape.k,
+            "n_init": shape.n_init, "n_local": shape.n_local, "l_c1": shape.l_c1,
+            "s_c1": shape.s_c1, "pool_l": shape.pool_l, "pool_s": shape.pool_s,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "no flush: Q (1.07 GB) alone exceeds the 126 MB L2"}
+
+
 def recorded_traffic(kernel: str):
     """DRAM bytes per unit from the committed ncu summary, if the kernel's
     source has not changed since the capture (else None)."""
@@ -297,12 +307,7 @@ def run_ours(args, rank, world, local_rank, dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) Q/V, K with per-block offsets and 128 planted needles)",
-        "config": {"workload": WORKLOAD, "n": n, "h_q": shape.h_q, "h_kv": shape.h_kv,
-                   "d": shape.d, "block": shape.B, "top_k_blocks": shape.k,
-                   "n_init": shape.n_init, "n_local": shape.n_local, "l_c1": shape.l_c1,
-                   "s_c1": shape.s_c1, "pool_l": shape.pool_l, "pool_s": shape.pool_s,
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "no flush: Q (1.07 GB) alone exceeds the 126 MB L2"},
+        "config": workload_config(shape, world),
         "tflops": round(tflops, 2),
         "tflops_frac_of_peak": round(tflops / world / peaks["bf16_tflops"], 4),
         "algorithmic_tflop_per_step": {"score": round(work["score"] / 1e12, 3),
@@ -687,7 +692,7 @@ def run_reference(args):
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * t_total / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "data": "synthetic", "config": workload_config(shape, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
