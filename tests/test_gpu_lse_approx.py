@@ -46,6 +46,7 @@ def test_compress_k2_bit_exact(n, h_kv):
     (600, 2, 2, 0, 600),          # G=1
     (900, 4, 2, 0, 900),          # G=2
     (20000, 16, 2, 19000, 1000),  # several coarse tiles
+    (100, 4, 1, 0, 100),          # shorter than one coarse kernel: every row exact
 ])
 def test_block_scores_approx_match_oracle(n, h_q, h_kv, q_begin, q_len):
     sh = synth.Shape(n=n, h_q=h_q, h_kv=h_kv, k=8)
