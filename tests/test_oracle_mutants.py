@@ -2,16 +2,36 @@
 
 Each mutant is a one-line textual change to oracle.c (a dropped term, a wrong
 index or sign, a swapped operand), compiled to a temporary library on the CPU.
+The pins run against each mutant in a child process: a mutant that writes out
+of bounds (k_excludes_forced fills more than k slots) may corrupt memory, and
+that must not take the test session down with it.
 """
 import os
 import subprocess
+import sys
 
 import pytest
 
 import oracle
-import pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+TESTS = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(TESTS)
+
+# Runs every pin against the library in argv[1] until one fails; prints the
+# name of each pin that failed its assertions.
+CHILD = """
+import sys
+sys.path[:0] = [%r, %r]
+import oracle, pins
+with oracle.use(oracle.load(sys.argv[1])):
+    for pin in pins.ALL_PINS:
+        try:
+            pin()
+        except AssertionError:
+            print("CAUGHT", pin.__name__, flush=True)
+            break
+"""
 
 MUTANTS = {
     "visibility_off_by_one": ("j * p->s_c1 + p->l_c1 - 1 <= i; ++j", "j * p->s_c1 + p->l_c1 <= i; ++j"),
@@ -36,22 +56,56 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutant_is_caught(name, tmp_path):
+def _mutant_source(name):
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
-    mutated = src.replace(old, new, 1)
-    c = tmp_path / "oracle_mut.c"
-    c.write_text(mutated)
-    so = tmp_path / "liboracle_mut.so"
-    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(c), "-o", str(so), "-lm"])
-    handle = oracle.load(str(so))
-    caught = []
-    with oracle.use(handle):
-        for pin in pins.ALL_PINS:
-            try:
-                pin()
-            except AssertionError:
-                caught.append(pin.__name__)
-    assert caught, f"no pin caught mutant {name}"
+    return src.replace(old, new, 1)
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    """Compile every mutant and run the pins against each in its own child
+    process, a few at a time.  name -> (caught pin names, return code, stderr)."""
+    d = tmp_path_factory.mktemp("mutants")
+    jobs = []
+    for name in sorted(MUTANTS):
+        try:
+            src = _mutant_source(name)
+        except AssertionError as e:
+            jobs.append((name, None, str(e)))
+            continue
+        c = d / (name + ".c")
+        c.write_text(src)
+        so = d / ("lib" + name + ".so")
+        subprocess.check_call(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(c),
+                               "-o", str(so), "-lm"])
+        jobs.append((name, so, None))
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    width = max(1, min(8, (os.cpu_count() or 2) // 2))
+    out, running = {}, []
+    pending = list(jobs)
+    while pending or running:
+        while pending and len(running) < width:
+            name, so, err = pending.pop(0)
+            if so is None:
+                out[name] = ([], None, err)
+                continue
+            proc = subprocess.Popen([sys.executable, "-c", CHILD % (ROOT, TESTS), str(so)],
+                                    stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True,
+                                    env=env)
+            running.append((name, proc))
+        if running:
+            name, proc = running.pop(0)
+            stdout, stderr = proc.communicate(timeout=600)
+            caught = [ln.split()[1] for ln in stdout.splitlines() if ln.startswith("CAUGHT ")]
+            out[name] = (caught, proc.returncode, stderr)
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, outcomes):
+    caught, rc, stderr = outcomes[name]
+    assert rc is not None, stderr                 # the mutation site exists
+    # a pin's failed assertion, or else the mutant crashing the oracle under a pin
+    assert caught or rc < 0, f"no pin caught mutant {name}: {stderr[-2000:]}"
