@@ -267,7 +267,7 @@ def run_ours(args, rank, world, local_rank, dist):
     approx = _lse_approx_timing(args, infv2, torch, shape, q, k, v, o, lse, stream, ms)
     bwd = _backward_timing(args, infv2, torch, p, shape, q, k, v, ws, stream)
     # ---- end to end through host buffers
-    e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_ranks)
+    e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_ranks)
     # ---- decode
     dec = _decode(args, infv2, torch, shape, rank, dev, stream, max_ranks, DecodeState)
     if infv2.infv2_device_status() != 0:
@@ -510,73 +510,43 @@ def _backward_timing(args, infv2, torch, p, shape, q, k, v, ws, stream):
             "note": "dq, dk, dv in fp32 over the prefill's block lists (selection fixed)"}
 
 
-def _end_to_end(args, infv2, torch, p, shape, data, cu, ws, stream, dev, max_over_ranks):
-    """Same metric through the C ABI with host buffers: every step copies its
-    inputs from pinned host memory and reads its output back.  The copies run
-    on their own streams, double-buffered, so that step j+1's inputs travel
-    and step j-1's output returns while step j computes (as a serving loop
-    would pipeline them); every copy of every timed step is inside the timed
-    region."""
+def _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_over_ranks):
+    """Same metric through the C ABI with host buffers (infv2_pipeline_*):
+    every step copies its inputs from pinned host memory and reads its output
+    back.  The library's pipeline copies on its own two streams into two
+    device slots, so that step j+1's inputs travel and step j-1's output
+    returns while step j computes (as a serving loop would pipeline them);
+    every copy of every timed step is inside the timed region."""
     qh = torch.from_numpy(data["q"].view(np.int16)).pin_memory()
     kh = torch.from_numpy(data["k"].view(np.int16)).pin_memory()
     vh = torch.from_numpy(data["v"].view(np.int16)).pin_memory()
     ohs = [torch.empty_like(qh).pin_memory() for _ in range(2)]
-    bufs = [dict(q=torch.empty(qh.shape, dtype=torch.int16, device=dev),
-                 k=torch.empty(kh.shape, dtype=torch.int16, device=dev),
-                 v=torch.empty(vh.shape, dtype=torch.int16, device=dev),
-                 o=torch.empty(qh.shape, dtype=torch.int16, device=dev)) for _ in range(2)]
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev = lambda: torch.cuda.Event()
-    in_done = [ev(), ev()]
-    comp_done = [ev(), ev()]
-    out_done = [ev(), ev()]
-    used = [False, False]
-
-    def step(j):
-        b = j % 2
-        buf = bufs[b]
-        with torch.cuda.stream(s_in):        # inputs of step j (after step j-2 read them)
-            if used[b]:
-                s_in.wait_event(comp_done[b])
-            buf["q"].copy_(qh, non_blocking=True)
-            buf["k"].copy_(kh, non_blocking=True)
-            buf["v"].copy_(vh, non_blocking=True)
-            in_done[b].record(s_in)
-        stream.wait_event(in_done[b])        # compute (after step j-2's output left)
-        if used[b]:
-            stream.wait_event(out_done[b])
-        infv2.infv2_prefill(p, buf["q"].view(torch.bfloat16), buf["k"].view(torch.bfloat16),
-                            buf["v"].view(torch.bfloat16), cu, workspace=ws,
-                            o=buf["o"].view(torch.bfloat16), stream=stream)
-        comp_done[b].record(stream)
-        with torch.cuda.stream(s_out):       # output of step j
-            s_out.wait_event(comp_done[b])
-            ohs[b].copy_(buf["o"], non_blocking=True)
-            out_done[b].record(s_out)
-        used[b] = True
-
-    for j in range(2):
-        step(j)
-    torch.cuda.synchronize()
-    steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
-    for j in range(steps):
-        step(2 + j)
-    stream.wait_stream(s_in)
-    stream.wait_stream(s_out)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    pl = infv2.infv2_pipeline_create(p, cu, stream=stream, device=dev)
+    try:
+        for j in range(2):
+            infv2.infv2_pipeline_submit(pl, qh, kh, vh, ohs[j % 2])
+        infv2.infv2_pipeline_sync(pl)
+        steps = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        infv2.infv2_pipeline_wait(pl, stream)
+        for j in range(steps):
+            infv2.infv2_pipeline_submit(pl, qh, kh, vh, ohs[j % 2])
+        infv2.infv2_pipeline_join(pl, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        infv2.infv2_pipeline_sync(pl)
+    finally:
+        infv2.infv2_pipeline_destroy(pl)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps)
     h2d = qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2
     d2h = ohs[0].numel() * 2
     world = int(os.environ.get("WORLD_SIZE", "1"))
     return {"value": round(job_throughput(world, shape.n, ms), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "overlap": "inputs of step j+1 and output of step j-1 copied on their own streams "
-                       "while step j computes (double-buffered)"}
+            "api": "infv2_pipeline_submit (host buffers)",
+            "overlap": "inputs of step j+1 and output of step j-1 copied on the pipeline's own "
+                       "streams while step j computes (two device slots)"}
 
 
 def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, DecodeState):

@@ -22,9 +22,10 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, unless a
- *     parameter says "host".  The library allocates no memory; scratch space
- *     is the caller's `workspace` (infv2_select_blocks_noalloc instead uses a
- *     fixed array that the library holds on each device).
+ *     parameter says "host".  The library allocates no device memory; scratch
+ *     space is the caller's `workspace` (infv2_select_blocks_noalloc instead
+ *     uses a fixed array that the library holds on each device; a pipeline
+ *     handle owns host state, two streams and events).
  *   - bf16 tensors are raw 16-bit patterns (e.g. torch.bfloat16 storage);
  *     every tensor is dense, row-major, 16-byte aligned.
  *   - Token layout ("thd"): q [n, h_q, d], k and v [n, h_kv, d]; query head h
@@ -33,8 +34,10 @@
  *     stream) and return an infv2_status for argument / launch errors.  Errors
  *     detected inside a kernel (a bounded wait that timed out) are recorded in
  *     a per-device word read by infv2_device_status().
- *   - No call retains a pointer after it returns; calls that share output or
- *     workspace memory must be ordered on the caller's streams.
+ *   - No call retains a pointer after it returns, except a pipeline, which
+ *     keeps its workspace and the host buffers of queued batches; calls that
+ *     share output or workspace memory must be ordered on the caller's
+ *     streams.
  */
 #ifndef INFV2_H
 #define INFV2_H
@@ -240,6 +243,72 @@ int infv2_prefill_workspace_size(const infv2_params* p, const int* cu_seqlens_ho
 int infv2_prefill(const infv2_params* p, const void* q, const void* k, const void* v,
                   const int* cu_seqlens_host, int batch, void* workspace, size_t ws_bytes,
                   int* idx_out, void* o, float* lse, infv2_stream_t stream);
+
+/* ---- Prefill over HOST buffers: a two-slot copy/compute pipeline ----------
+ * The same layer as infv2_prefill for a serving loop whose Q, K, V arrive in
+ * host memory and whose O must return there.  A pipeline is bound to one
+ * varlen shape (cu_seqlens) and one device (the current one at creation).
+ * Each submit takes one of two device slots in turn:
+ *   - its inputs are copied host -> device on the pipeline's input stream;
+ *   - infv2_prefill runs on the caller's compute stream;
+ *   - O (and the log-sum-exp) are copied device -> host on its output stream.
+ * With page-locked host buffers, batch j+1's inputs and batch j-1's output
+ * cross PCIe while batch j computes; pageable buffers are accepted but their
+ * copies serialise with the host.  Slot reuse is ordered by events, so any
+ * number of submits may be queued.  The library allocates no device memory
+ * for a pipeline: the caller's workspace holds the prefill workspace and both
+ * slots.  The pipeline owns two CUDA streams and seven events, released by
+ * infv2_pipeline_destroy. */
+typedef struct infv2_pipeline infv2_pipeline;
+
+/* Device workspace bytes a pipeline for this varlen batch needs: the
+ * infv2_prefill workspace plus, per slot, q, k, v, o and lse.
+ * cu_seqlens_host: HOST int32 [batch + 1], cu_seqlens_host[0] = 0, batch >= 1,
+ * at least one token.  Host-only; INFV2_ERR_INVALID_ARG on bad shapes. */
+int infv2_pipeline_workspace_size(const infv2_params* p, const int* cu_seqlens_host, int batch,
+                                  size_t* bytes);
+
+/* Create a pipeline on the current device.
+ *   workspace  device memory of at least infv2_pipeline_workspace_size bytes,
+ *              256-byte aligned, owned by the caller and kept alive and
+ *              untouched until infv2_pipeline_destroy returns;
+ *   stream     the compute stream (the prefill kernels run there);
+ *   *out       receives the handle (NULL on failure).
+ * Errors: INFV2_ERR_INVALID_ARG (bad shape, NULL or misaligned workspace),
+ * INFV2_ERR_WORKSPACE (too small), INFV2_ERR_CUDA (a stream or event could
+ * not be created, or host memory ran out). */
+int infv2_pipeline_create(const infv2_params* p, const int* cu_seqlens_host, int batch,
+                          void* workspace, size_t ws_bytes, infv2_stream_t stream,
+                          infv2_pipeline** out);
+
+/* Enqueue one batch and return without waiting.
+ *   q_host  HOST bf16 [T, h_q, d];  k_host, v_host  HOST bf16 [T, h_kv, d]
+ *   o_host  HOST bf16 [T, h_q, d] (output)
+ *   lse_host  HOST fp32 [h_q, T] (output, nullable)
+ * T = cu_seqlens_host[batch] of the pipeline.  The host buffers must stay
+ * allocated and the inputs unchanged, and the outputs must not be read, until
+ * infv2_pipeline_sync returns (or a stream given to infv2_pipeline_join has
+ * passed that point).  Errors: INFV2_ERR_INVALID_ARG (NULL pointer),
+ * INFV2_ERR_CUDA (a copy, event or launch failed; the pipeline should then
+ * be destroyed). */
+int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, const void* k_host,
+                          const void* v_host, void* o_host, float* lse_host);
+
+/* Order the work submitted after this call behind the work enqueued so far on
+ * `stream` (all three of the pipeline's streams wait for it). */
+int infv2_pipeline_wait(infv2_pipeline* pl, infv2_stream_t stream);
+
+/* Make `stream` wait, without blocking the host, until every batch submitted
+ * so far has landed in its host output buffers. */
+int infv2_pipeline_join(infv2_pipeline* pl, infv2_stream_t stream);
+
+/* Block the host until every batch submitted so far has landed in its host
+ * output buffers.  INFV2_ERR_CUDA if a copy or kernel failed. */
+int infv2_pipeline_sync(infv2_pipeline* pl);
+
+/* Wait for the pipeline's streams, release them and the events, and free the
+ * handle (NULL is a no-op).  The workspace may be freed afterwards. */
+int infv2_pipeline_destroy(infv2_pipeline* pl);
 
 /* Workspace bytes that infv2_decode needs. */
 int infv2_decode_workspace_size(const infv2_params* p, int batch, int cap, size_t* bytes);

@@ -125,3 +125,53 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_block_scores_approx(P, None, None, None, 100, 50, 60, None, 128, None, None) == infv2.ERR_INVALID_ARG
     assert L.infv2_prefill_workspace_size(ctypes.byref(pa), (ctypes.c_int * 2)(0, 10000), 1, ctypes.byref(sz)) == infv2.OK
     assert L.infv2_check_params(None) == infv2.ERR_INVALID_ARG
+
+
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_pipeline_workspace_and_argument_errors():
+    L = infv2.lib()
+    p = infv2.params(32, 2)
+    P = ctypes.byref(p)
+    for cu in ([0, 131072], [0, 300, 5000, 5001]):
+        T = cu[-1]
+        q, kv, lse = T * 32 * 128 * 2, T * 2 * 128 * 2, T * 32 * 4
+        slot = 2 * _r256(q) + 2 * _r256(kv) + _r256(lse)
+        want = _r256(infv2.infv2_prefill_workspace_size(p, cu)) + 2 * slot
+        assert infv2.infv2_pipeline_workspace_size(p, cu) == want
+    sz = ctypes.c_size_t()
+    cu = (ctypes.c_int * 3)(0, 100, 300)
+    assert L.infv2_pipeline_workspace_size(P, cu, 0, ctypes.byref(sz)) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_workspace_size(P, (ctypes.c_int * 2)(0, 0), 1, ctypes.byref(sz)) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_workspace_size(P, (ctypes.c_int * 2)(4, 9), 1, ctypes.byref(sz)) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_workspace_size(P, cu, 2, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_workspace_size(P, cu, 2, ctypes.byref(sz)) == infv2.OK
+    h = ctypes.c_void_p()
+    # every argument error is caught before the workspace is touched or CUDA is called
+    assert L.infv2_pipeline_create(P, cu, 2, 4096, sz.value, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_create(P, cu, 2, None, sz.value, None, ctypes.byref(h)) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_create(P, cu, 2, 4096 + 16, sz.value, None, ctypes.byref(h)) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_create(P, cu, 2, 4096, sz.value - 1, None, ctypes.byref(h)) == infv2.ERR_WORKSPACE
+    assert not h.value
+    assert L.infv2_pipeline_submit(None, 16, 16, 16, 16, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_wait(None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_join(None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_sync(None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_pipeline_destroy(None) == infv2.OK
+
+
+def test_pipeline_binding_checks_host_buffer_sizes():
+    import torch
+    p = infv2.params(4, 1)
+    pl = infv2.Pipeline(ctypes.c_void_p(), None, p, [0, 100], None)   # no handle: nothing is called
+    q = torch.zeros((100, 4, 128), dtype=torch.bfloat16)
+    kv = torch.zeros((100, 1, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        infv2.infv2_pipeline_submit(pl, q[:99], kv, kv, q)
+    with pytest.raises(ValueError):
+        infv2.infv2_pipeline_submit(pl, q, kv, kv, q, torch.zeros((4, 99)))
+    with pytest.raises(ValueError):
+        infv2.infv2_pipeline_submit(pl, q, torch.zeros((100, 2, 128), dtype=torch.bfloat16)[:, :1], kv, q)
+    infv2.infv2_pipeline_destroy(pl)   # a handle that was never created: no-op

@@ -24,7 +24,9 @@ SYMBOLS = [
     "infv2_decode_workspace_size", "infv2_decode", "infv2_select_blocks_noalloc",
     "infv2_selftest_timeout", "infv2_block_scores_pooled", "infv2_select_topk_pooled",
     "infv2_compress_k2", "infv2_block_scores_approx", "infv2_sparse_attn_bwd_workspace_size",
-    "infv2_sparse_attn_bwd",
+    "infv2_sparse_attn_bwd", "infv2_pipeline_workspace_size", "infv2_pipeline_create",
+    "infv2_pipeline_submit", "infv2_pipeline_wait", "infv2_pipeline_join", "infv2_pipeline_sync",
+    "infv2_pipeline_destroy",
 ]
 
 
@@ -78,6 +80,13 @@ def lib():
         L.infv2_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i, i, vp, sz, vp, vp, vp, vp]
         L.infv2_select_blocks_noalloc.argtypes = [P, vp, vp, i, i, i, vp, vp]
         L.infv2_selftest_timeout.argtypes = [i, vp]
+        L.infv2_pipeline_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
+        L.infv2_pipeline_create.argtypes = [P, vp, i, vp, sz, vp, ctypes.POINTER(vp)]
+        L.infv2_pipeline_submit.argtypes = [vp, vp, vp, vp, vp, vp]
+        L.infv2_pipeline_wait.argtypes = [vp, vp]
+        L.infv2_pipeline_join.argtypes = [vp, vp]
+        L.infv2_pipeline_sync.argtypes = [vp]
+        L.infv2_pipeline_destroy.argtypes = [vp]
         _lib = L
     return _lib
 
@@ -292,6 +301,86 @@ def infv2_prefill(p: Params, q, k, v, cu_seqlens, workspace=None, idx_out=None, 
                                _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(o),
                                _ptr(lse), _stream(stream)), "infv2_prefill")
     return o
+
+
+def _cu_array(cu_seqlens):
+    return (ctypes.c_int * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+
+
+def _host_ptr(t, nbytes: int, what: str):
+    """Address of a contiguous host tensor of exactly nbytes (None passes)."""
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s: expected a contiguous host tensor" % what)
+    if t.numel() * t.element_size() != nbytes:
+        raise ValueError("%s: %d bytes, the pipeline's shape needs %d"
+                         % (what, t.numel() * t.element_size(), nbytes))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Pipeline:
+    """Handle of an infv2_pipeline (the device workspace it keeps alive, and
+    the varlen shape it was created for)."""
+
+    def __init__(self, handle, workspace, p: Params, cu_seqlens, stream):
+        self.handle, self.workspace, self.stream = handle, workspace, stream
+        T = int(cu_seqlens[-1])
+        self.q_bytes = T * p.h_q * p.d * 2
+        self.kv_bytes = T * p.h_kv * p.d * 2
+        self.lse_bytes = T * p.h_q * 4
+
+
+def infv2_pipeline_workspace_size(p: Params, cu_seqlens) -> int:
+    cu = _cu_array(cu_seqlens)
+    out = ctypes.c_size_t(0)
+    _check(lib().infv2_pipeline_workspace_size(ctypes.byref(p), ctypes.cast(cu, ctypes.c_void_p),
+                                               len(cu_seqlens) - 1, ctypes.byref(out)),
+           "infv2_pipeline_workspace_size")
+    return out.value
+
+
+def infv2_pipeline_create(p: Params, cu_seqlens, workspace=None, stream=None,
+                          device=None) -> Pipeline:
+    """Pipeline for prefill over host buffers; `stream` is the compute stream."""
+    need = infv2_pipeline_workspace_size(p, cu_seqlens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device or "cuda")
+    cu = _cu_array(cu_seqlens)
+    h = ctypes.c_void_p()
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check(lib().infv2_pipeline_create(ctypes.byref(p), ctypes.cast(cu, ctypes.c_void_p),
+                                       len(cu_seqlens) - 1, _ptr(workspace), workspace.numel(),
+                                       _stream(s), ctypes.byref(h)), "infv2_pipeline_create")
+    return Pipeline(h, workspace, p, cu_seqlens, s)
+
+
+def infv2_pipeline_submit(pl: Pipeline, q_host, k_host, v_host, o_host, lse_host=None):
+    """Queue one batch: host bf16 q/k/v in, host bf16 o (and fp32 lse) out."""
+    _check(lib().infv2_pipeline_submit(pl.handle, _host_ptr(q_host, pl.q_bytes, "q_host"),
+                                       _host_ptr(k_host, pl.kv_bytes, "k_host"),
+                                       _host_ptr(v_host, pl.kv_bytes, "v_host"),
+                                       _host_ptr(o_host, pl.q_bytes, "o_host"),
+                                       _host_ptr(lse_host, pl.lse_bytes, "lse_host")),
+           "infv2_pipeline_submit")
+
+
+def infv2_pipeline_wait(pl: Pipeline, stream=None):
+    _check(lib().infv2_pipeline_wait(pl.handle, _stream(stream)), "infv2_pipeline_wait")
+
+
+def infv2_pipeline_join(pl: Pipeline, stream=None):
+    _check(lib().infv2_pipeline_join(pl.handle, _stream(stream)), "infv2_pipeline_join")
+
+
+def infv2_pipeline_sync(pl: Pipeline):
+    _check(lib().infv2_pipeline_sync(pl.handle), "infv2_pipeline_sync")
+
+
+def infv2_pipeline_destroy(pl: Pipeline):
+    if pl.handle is not None and pl.handle.value:
+        h, pl.handle = pl.handle, None
+        _check(lib().infv2_pipeline_destroy(h), "infv2_pipeline_destroy")
 
 
 def infv2_decode_workspace_size(p: Params, batch: int, cap: int) -> int:
