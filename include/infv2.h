@@ -250,15 +250,19 @@ int infv2_prefill(const infv2_params* p, const void* q, const void* k, const voi
  * varlen shape (cu_seqlens) and one device (the current one at creation).
  * Each submit takes one of two device slots in turn:
  *   - its inputs are copied host -> device on the pipeline's input stream;
- *   - infv2_prefill runs on the caller's compute stream;
+ *   - the prefill runs on the caller's compute stream;
  *   - O (and the log-sum-exp) are copied device -> host on its output stream.
  * With page-locked host buffers, batch j+1's inputs and batch j-1's output
  * cross PCIe while batch j computes; pageable buffers are accepted but their
- * copies serialise with the host.  Slot reuse is ordered by events, so any
- * number of submits may be queued.  The library allocates no device memory
- * for a pipeline: the caller's workspace holds the prefill workspace and both
- * slots.  The pipeline owns two CUDA streams and seven events, released by
- * infv2_pipeline_destroy. */
+ * copies serialise with the host.  Within a batch, K and V are copied first
+ * and Q in parts of 8192 tokens; each score chunk waits only for the Q rows it
+ * reads, the attention runs in row ranges between the score chunks, and each
+ * finished range of O (and its log-sum-exp) is copied back while the next
+ * range computes.  The results are those of infv2_prefill, bit for bit.
+ * Slot reuse is ordered by events, so any number of submits may be queued.
+ * The library allocates no device memory for a pipeline: the caller's
+ * workspace holds the prefill workspace and both slots.  The pipeline owns
+ * two CUDA streams and its events, released by infv2_pipeline_destroy. */
 typedef struct infv2_pipeline infv2_pipeline;
 
 /* Device workspace bytes a pipeline for this varlen batch needs: the

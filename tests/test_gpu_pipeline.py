@@ -32,10 +32,16 @@ def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("lengths", [[700, 300, 5000, 1300], [2048]])
-def test_pipeline_matches_device_prefill_and_oracle(lengths):
-    # k*B = 512: the 300-token sequence is dense, the others sparse
-    sh = synth.Shape(n=0, h_q=16, h_kv=2, k=8)
+@pytest.mark.parametrize("lengths,h_q,h_kv", [
+    ([700, 300, 5000, 1300], 16, 2),
+    ([2048], 16, 2),
+    # 20000 tokens at h_kv = 8: four score chunks, so the attention runs as four
+    # row ranges between them (the single-launch device prefill is the reference)
+    ([20000, 300], 16, 8),
+])
+def test_pipeline_matches_device_prefill_and_oracle(lengths, h_q, h_kv):
+    # k*B = 512: 300-token sequences are dense, the others sparse
+    sh = synth.Shape(n=0, h_q=h_q, h_kv=h_kv, k=8)
     sets = [synth.make_varlen(sh, lengths, seed=s, n_needles=2) for s in range(3)]
     cu = [int(x) for x in sets[0]["cu_seqlens"]]
     T = cu[-1]

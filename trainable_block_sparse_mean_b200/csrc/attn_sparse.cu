@@ -77,7 +77,7 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, long long w) {
   const long long per_g = (long long)a.n_rows * a.n_split;
   it.g = (int)(w / per_g);
   const long long rem = w % per_g;
-  it.r = (int)(rem / a.n_split);
+  it.r = a.row_begin + (int)(rem / a.n_split);
   it.sp = (int)(rem % a.n_split);
   return it;
 }
@@ -520,7 +520,8 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
   if (n_items == 0) return INFV2_OK;
   const int G = a.h_q / a.h_kv;
   CUtensorMap tm_q;  // q [rows, h_q, 128]: one item = G heads of one row
-  if (!make_tmap_3d(&tm_q, a.q, 128, a.h_q, a.n_rows, 256, (uint64_t)a.h_q * 256, 64, G, 1))
+  if (!make_tmap_3d(&tm_q, a.q, 128, a.h_q, a.row_begin + a.n_rows, 256, (uint64_t)a.h_q * 256,
+                    64, G, 1))
     return INFV2_ERR_CUDA;
   const int smem = kStages * kStageBytes + (4 * 16 * 128 + 128) * 4 + 2 * kQSlot +
                    8 * (2 * kStages + 1 + 4) + 1024;
@@ -536,16 +537,19 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
 }
 
 // Prefill form: K/V [n, h_kv, 128], idx [h_kv, n, k] with the given strides.
-int launch_sparse_attn_prefill(const infv2_params* p, const uint16_t* q, const uint16_t* k,
-                               const uint16_t* v, const int* idx, long long idx_hstride, int n,
-                               uint16_t* o, float* lse, long long lse_ld, cudaStream_t st) {
-  if (n <= 0) return INFV2_OK;
+int launch_sparse_attn_rows(const infv2_params* p, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const int* idx, long long idx_hstride, int n,
+                            int r0, int r1, uint16_t* o, float* lse, long long lse_ld,
+                            cudaStream_t st) {
+  if (r0 < 0 || r1 > n || r0 > r1) return INFV2_ERR_INVALID_ARG;
+  if (r1 == r0) return INFV2_OK;
   CUtensorMap tm_k, tm_v;
   if (!make_tmap_3d(&tm_k, k, 128, p->h_kv, n, 256, (uint64_t)p->h_kv * 256, 64, 1, 64) ||
       !make_tmap_3d(&tm_v, v, 128, p->h_kv, n, 256, (uint64_t)p->h_kv * 256, 64, 1, 64))
     return INFV2_ERR_CUDA;
   AttnArgs a{};
-  a.n_rows = n;
+  a.n_rows = r1 - r0;
+  a.row_begin = r0;
   a.h_q = p->h_q;
   a.h_kv = p->h_kv;
   a.k = p->k;
@@ -563,6 +567,13 @@ int launch_sparse_attn_prefill(const infv2_params* p, const uint16_t* q, const u
   a.split_out = 0;
   a.wait = wait_ctx();
   return launch_sparse_attn(tm_k, tm_v, a, st);
+}
+
+int launch_sparse_attn_prefill(const infv2_params* p, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const int* idx, long long idx_hstride, int n,
+                               uint16_t* o, float* lse, long long lse_ld, cudaStream_t st) {
+  if (n <= 0) return INFV2_OK;
+  return launch_sparse_attn_rows(p, q, k, v, idx, idx_hstride, n, 0, n, o, lse, lse_ld, st);
 }
 
 }  // namespace infv2

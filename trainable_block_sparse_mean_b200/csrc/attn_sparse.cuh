@@ -6,6 +6,8 @@ namespace infv2 {
 
 struct AttnArgs {
   int n_rows;              // prefill: tokens of the sequence; decode: sequences of the batch
+  int row_begin;           // prefill: first query row of this launch (rows row_begin ..
+                           // row_begin + n_rows - 1); decode: 0
   int h_q, h_kv, k;
   const int* idx;          // block list of (g, row): idx + g*idx_hstride + row*idx_rstride
   long long idx_hstride, idx_rstride;
@@ -33,6 +35,13 @@ int launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const A
 int launch_sparse_attn_prefill(const infv2_params* p, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int* idx, long long idx_hstride, int n,
                                uint16_t* o, float* lse, long long lse_ld, cudaStream_t st);
+
+// The same over query rows [r0, r1) of the n-token sequence only (q, k, v, idx,
+// o and lse are the whole sequence's; rows outside the range are not touched).
+int launch_sparse_attn_rows(const infv2_params* p, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const int* idx, long long idx_hstride, int n,
+                            int r0, int r1, uint16_t* o, float* lse, long long lse_ld,
+                            cudaStream_t st);
 
 }  // namespace infv2
 

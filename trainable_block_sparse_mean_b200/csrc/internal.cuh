@@ -46,4 +46,23 @@ inline int shared_ld(int n) {
 
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Hooks of a staged prefill (the host-buffer pipeline).  need_q(t_end) runs on
+// the host before the first launch that reads packed query rows below t_end;
+// done_o(t0, t1) right after the launch that completes output rows [t0, t1).
+// Both may enqueue stream waits or event records; a non-zero status aborts.
+struct PrefillHooks {
+  int attn_parts = 1;  // attention launches per sparse sequence (row ranges)
+  virtual int need_q(long long t_end) = 0;
+  virtual int done_o(long long t0, long long t1) = 0;
+
+ protected:
+  ~PrefillHooks() = default;
+};
+
+// The whole layer over a packed varlen batch (infv2_prefill's body); hooks may
+// be null.  Without hooks the launch sequence is exactly infv2_prefill's.
+int run_prefill(const infv2_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const int* cu_seqlens_host, int batch, void* workspace, size_t ws_bytes,
+                int* idx_out, uint16_t* o, float* lse, cudaStream_t st, PrefillHooks* hooks);
+
 }  // namespace infv2

@@ -5,10 +5,14 @@
 // cross to the device on the pipeline's input stream, the whole prefill runs
 // on the caller's compute stream, and O (and the log-sum-exp) return on the
 // output stream.  With page-locked host buffers the inputs of batch j+1 and
-// the output of batch j-1 travel while batch j computes.  Slot reuse is
-// ordered by events: a slot's inputs are overwritten only after the compute
-// of the batch two submits earlier has read them, and its output only after
-// that batch's output has left.
+// the output of batch j-1 travel while batch j computes.  Within a batch the
+// copies are cut into parts as well: K and V first, then Q in parts of 8192
+// tokens, each score chunk waiting only for the Q rows it reads; the
+// attention runs in row ranges interleaved with the score chunks, and each
+// finished range of O leaves while the next computes.  Slot reuse is ordered
+// by events: a slot's inputs are overwritten only after the compute of the
+// batch two submits earlier has read them, and its output only after that
+// batch's output has left.
 #include <new>
 #include <vector>
 
@@ -16,6 +20,10 @@
 
 namespace infv2 {
 namespace {
+
+constexpr int kQPartRows = 8192;                     // tokens per host->device Q copy
+constexpr size_t kOutFlushBytes = size_t(64) << 20;  // output copies coalesced up to this
+constexpr int kAttnParts = 8;                        // attention row ranges per sequence
 
 struct PipeLayout {
   size_t prefill_ws = 0;                  // workspace of infv2_prefill
@@ -80,12 +88,16 @@ struct infv2_pipeline {
   Slot slot[2];
   cudaStream_t compute = nullptr;  // the caller's stream
   cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t in_done[2] = {nullptr, nullptr};
+  cudaEvent_t in_done[2] = {nullptr, nullptr};  // K and V of the slot arrived
+  std::vector<cudaEvent_t> q_done[2];            // Q part i of the slot arrived
+  std::vector<cudaEvent_t> o_ready[2];           // a range of O computed (grown on demand)
   cudaEvent_t comp_done[2] = {nullptr, nullptr};
   cudaEvent_t out_done[2] = {nullptr, nullptr};
   cudaEvent_t fence = nullptr;
   bool used[2] = {false, false};
   int next = 0;
+  long long T = 0;
+  int n_qparts = 0;
 };
 
 namespace {
@@ -94,6 +106,9 @@ void release(infv2_pipeline* pl) {
   if (pl->s_in) cudaStreamSynchronize(pl->s_in);
   if (pl->s_out) cudaStreamSynchronize(pl->s_out);
   for (int b = 0; b < 2; ++b) {
+    for (cudaEvent_t e : pl->q_done[b])
+      if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : pl->o_ready[b]) cudaEventDestroy(e);
     if (pl->in_done[b]) cudaEventDestroy(pl->in_done[b]);
     if (pl->comp_done[b]) cudaEventDestroy(pl->comp_done[b]);
     if (pl->out_done[b]) cudaEventDestroy(pl->out_done[b]);
@@ -132,6 +147,8 @@ extern "C" int infv2_pipeline_create(const infv2_params* p, const int* cu_seqlen
   pl->cu.assign(cu_seqlens_host, cu_seqlens_host + batch + 1);
   pl->batch = batch;
   pl->L = L;
+  pl->T = cu_seqlens_host[batch];
+  pl->n_qparts = (int)((pl->T + kQPartRows - 1) / kQPartRows);
   pl->compute = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pl->prefill_ws = ws;
@@ -152,6 +169,9 @@ extern "C" int infv2_pipeline_create(const infv2_params* p, const int* cu_seqlen
   ok = ok && cudaStreamCreateWithFlags(&pl->s_in, cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaStreamCreateWithFlags(&pl->s_out, cudaStreamNonBlocking) == cudaSuccess;
   for (int b = 0; b < 2 && ok; ++b) {
+    pl->q_done[b].assign(pl->n_qparts, nullptr);
+    for (int i = 0; i < pl->n_qparts && ok; ++i)
+      ok = cudaEventCreateWithFlags(&pl->q_done[b][i], cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaEventCreateWithFlags(&pl->in_done[b], cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaEventCreateWithFlags(&pl->comp_done[b], cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaEventCreateWithFlags(&pl->out_done[b], cudaEventDisableTiming) == cudaSuccess;
@@ -171,6 +191,78 @@ extern "C" int infv2_pipeline_create(const infv2_params* p, const int* cu_seqlen
     if ((call) != cudaSuccess) return INFV2_ERR_CUDA; \
   } while (0)
 
+namespace {
+
+// The prefill's hooks for one submit: the compute stream waits for each Q part
+// before the first launch that reads it, and finished ranges of O (and the
+// log-sum-exp) are copied back on the output stream, coalesced up to
+// kOutFlushBytes.
+struct SubmitHooks final : PrefillHooks {
+  infv2_pipeline* pl;
+  int b;
+  uint16_t* o_host;
+  float* lse_host;
+  int q_waited = 0;
+  long long o_begin = 0, o_end = 0;  // computed output rows not yet copied back
+  int n_ready = 0;                   // o_ready events used by this submit
+
+  SubmitHooks(infv2_pipeline* pl_, int b_, void* o, float* lse)
+      : pl(pl_), b(b_), o_host(static_cast<uint16_t*>(o)), lse_host(lse) {
+    attn_parts = kAttnParts;
+  }
+
+  int need_q(long long t_end) override {
+    while (q_waited < pl->n_qparts && (long long)q_waited * kQPartRows < t_end) {
+      if (cudaStreamWaitEvent(pl->compute, pl->q_done[b][q_waited], 0) != cudaSuccess)
+        return INFV2_ERR_CUDA;
+      ++q_waited;
+    }
+    return INFV2_OK;
+  }
+
+  int done_o(long long t0, long long t1) override {
+    if (t0 != o_end) {  // not contiguous with the pending range: send that first
+      const int st = flush();
+      if (st != INFV2_OK) return st;
+      o_begin = t0;
+    }
+    o_end = t1;
+    const size_t row_bytes = (size_t)pl->p.h_q * pl->p.d * 2;
+    return (size_t)(o_end - o_begin) * row_bytes >= kOutFlushBytes ? flush() : INFV2_OK;
+  }
+
+  int flush() {
+    if (o_end <= o_begin) return INFV2_OK;
+    std::vector<cudaEvent_t>& ev = pl->o_ready[b];
+    if (n_ready == (int)ev.size()) {
+      cudaEvent_t e;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return INFV2_ERR_CUDA;
+      ev.push_back(e);
+    }
+    cudaEvent_t e = ev[n_ready++];
+    const Slot& s = pl->slot[b];
+    const size_t row_bytes = (size_t)pl->p.h_q * pl->p.d * 2;
+    if (cudaEventRecord(e, pl->compute) != cudaSuccess ||
+        cudaStreamWaitEvent(pl->s_out, e, 0) != cudaSuccess ||
+        cudaMemcpyAsync(reinterpret_cast<uint8_t*>(o_host) + o_begin * row_bytes,
+                        reinterpret_cast<const uint8_t*>(s.o) + o_begin * row_bytes,
+                        (size_t)(o_end - o_begin) * row_bytes, cudaMemcpyDeviceToHost,
+                        pl->s_out) != cudaSuccess)
+      return INFV2_ERR_CUDA;
+    if (lse_host) {  // lse [h_q, T]: the range is one strip per head
+      const size_t pitch = (size_t)pl->T * 4;
+      if (cudaMemcpy2DAsync(lse_host + o_begin, pitch, s.lse + o_begin, pitch,
+                            (size_t)(o_end - o_begin) * 4, pl->p.h_q, cudaMemcpyDeviceToHost,
+                            pl->s_out) != cudaSuccess)
+        return INFV2_ERR_CUDA;
+    }
+    o_begin = o_end;
+    return INFV2_OK;
+  }
+};
+
+}  // namespace
+
 extern "C" int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, const void* k_host,
                                      const void* v_host, void* o_host, float* lse_host) {
   if (!pl || !q_host || !k_host || !v_host || !o_host) return INFV2_ERR_INVALID_ARG;
@@ -179,25 +271,31 @@ extern "C" int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, con
   const int b = pl->next;
   const Slot& s = pl->slot[b];
   const PipeLayout& L = pl->L;
-  // inputs: after the compute of the batch two submits back has read this slot
+  // inputs: after the compute of the batch two submits back has read this slot;
+  // K and V first (compression and attention need all of them), then Q in parts
   if (pl->used[b]) PIPE_CK(cudaStreamWaitEvent(pl->s_in, pl->comp_done[b], 0));
-  PIPE_CK(cudaMemcpyAsync(s.q, q_host, L.q_bytes, cudaMemcpyHostToDevice, pl->s_in));
   PIPE_CK(cudaMemcpyAsync(s.k, k_host, L.kv_bytes, cudaMemcpyHostToDevice, pl->s_in));
   PIPE_CK(cudaMemcpyAsync(s.v, v_host, L.kv_bytes, cudaMemcpyHostToDevice, pl->s_in));
   PIPE_CK(cudaEventRecord(pl->in_done[b], pl->s_in));
-  // compute: after this batch's inputs arrived and the slot's previous output left
+  const size_t q_row = (size_t)pl->p.h_q * pl->p.d * 2;
+  for (int i = 0; i < pl->n_qparts; ++i) {
+    const long long t0 = (long long)i * kQPartRows;
+    const long long t1 = t0 + kQPartRows < pl->T ? t0 + kQPartRows : pl->T;
+    PIPE_CK(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(s.q) + t0 * q_row,
+                            static_cast<const uint8_t*>(q_host) + t0 * q_row,
+                            (size_t)(t1 - t0) * q_row, cudaMemcpyHostToDevice, pl->s_in));
+    PIPE_CK(cudaEventRecord(pl->q_done[b][i], pl->s_in));
+  }
+  // compute: after this batch's K/V arrived and the slot's previous output left
   PIPE_CK(cudaStreamWaitEvent(pl->compute, pl->in_done[b], 0));
   if (pl->used[b]) PIPE_CK(cudaStreamWaitEvent(pl->compute, pl->out_done[b], 0));
-  const int st = infv2_prefill(&pl->p, s.q, s.k, s.v, pl->cu.data(), pl->batch, pl->prefill_ws,
-                               L.prefill_ws, nullptr, s.o, lse_host ? s.lse : nullptr,
-                               reinterpret_cast<infv2_stream_t>(pl->compute));
+  SubmitHooks hooks(pl, b, o_host, lse_host);
+  int st = run_prefill(&pl->p, s.q, s.k, s.v, pl->cu.data(), pl->batch, pl->prefill_ws,
+                       L.prefill_ws, nullptr, s.o, lse_host ? s.lse : nullptr, pl->compute, &hooks);
+  if (st == INFV2_OK) st = hooks.need_q(pl->T);  // every Q part before comp_done
+  if (st == INFV2_OK) st = hooks.flush();
   if (st != INFV2_OK) return st;
   PIPE_CK(cudaEventRecord(pl->comp_done[b], pl->compute));
-  // outputs
-  PIPE_CK(cudaStreamWaitEvent(pl->s_out, pl->comp_done[b], 0));
-  PIPE_CK(cudaMemcpyAsync(o_host, s.o, L.q_bytes, cudaMemcpyDeviceToHost, pl->s_out));
-  if (lse_host)
-    PIPE_CK(cudaMemcpyAsync(lse_host, s.lse, L.lse_bytes, cudaMemcpyDeviceToHost, pl->s_out));
   PIPE_CK(cudaEventRecord(pl->out_done[b], pl->s_out));
   pl->used[b] = true;
   pl->next = b ^ 1;

@@ -74,38 +74,35 @@ extern "C" int infv2_prefill_workspace_size(const infv2_params* p, const int* cu
   return INFV2_OK;
 }
 
-extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k, const void* v,
-                             const int* cu_seqlens_host, int batch, void* workspace,
-                             size_t ws_bytes, int* idx_out, void* o, float* lse,
-                             infv2_stream_t stream) {
+namespace infv2 {
+
+int run_prefill(const infv2_params* p, const uint16_t* qb, const uint16_t* kb, const uint16_t* vb,
+                const int* cu, int batch, void* workspace, size_t ws_bytes, int* idx_out,
+                uint16_t* ob, float* lse, cudaStream_t cs, PrefillHooks* hooks) {
   int st = infv2_check_params(p);
   if (st != INFV2_OK) return st;
-  if (!cu_seqlens_host || batch < 0) return INFV2_ERR_INVALID_ARG;
+  if (!cu || batch < 0) return INFV2_ERR_INVALID_ARG;
   if (batch == 0) return INFV2_OK;
-  if (cu_seqlens_host[0] != 0) return INFV2_ERR_INVALID_ARG;
-  const long long T = cu_seqlens_host[batch];
+  if (cu[0] != 0) return INFV2_ERR_INVALID_ARG;
+  const long long T = cu[batch];
   if (T == 0) return INFV2_OK;
-  if (!q || !k || !v || !o) return INFV2_ERR_INVALID_ARG;
+  if (!qb || !kb || !vb || !ob) return INFV2_ERR_INVALID_ARG;
   PrefillPlan pl;
-  st = plan_prefill(p, cu_seqlens_host, batch, &pl);
+  st = plan_prefill(p, cu, batch, &pl);
   if (st != INFV2_OK) return st;
   if (pl.total > 0) {
     if (!workspace || ws_bytes < pl.total) return INFV2_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return INFV2_ERR_INVALID_ARG;
   }
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* kc1 = reinterpret_cast<uint16_t*>(ws + pl.off_kc1);
   uint16_t* kc2 = reinterpret_cast<uint16_t*>(ws + pl.off_kc2);
   float* s_shared = reinterpret_cast<float*>(ws + pl.off_shared);
   int* idx_ws = reinterpret_cast<int*>(ws + pl.off_idx);
-  const uint16_t* qb = static_cast<const uint16_t*>(q);
-  const uint16_t* kb = static_cast<const uint16_t*>(k);
-  const uint16_t* vb = static_cast<const uint16_t*>(v);
-  uint16_t* ob = static_cast<uint16_t*>(o);
+  const int parts = hooks && hooks->attn_parts > 1 ? hooks->attn_parts : 1;
   for (int s = 0; s < batch; ++s) {
-    const long long off = cu_seqlens_host[s];
-    const int n = cu_seqlens_host[s + 1] - cu_seqlens_host[s];
+    const long long off = cu[s];
+    const int n = cu[s + 1] - cu[s];
     if (n == 0) continue;
     const uint16_t* qs = qb + off * p->h_q * 128;
     const uint16_t* ks = kb + off * p->h_kv * 128;
@@ -113,8 +110,10 @@ extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k
     uint16_t* os = ob + off * p->h_q * 128;
     float* lses = lse ? lse + off : nullptr;
     if (n <= p->k * p->B) {
+      if (hooks && (st = hooks->need_q(off + n)) != INFV2_OK) return st;
       st = launch_dense_attn_blocks(p, qs, ks, vs, n, os, lses, T, cs);
       if (st != INFV2_OK) return st;
+      if (hooks && (st = hooks->done_o(off, off + n)) != INFV2_OK) return st;
       continue;
     }
     st = launch_compress_k(ks, n, p->h_kv, kc1, cs);
@@ -125,17 +124,39 @@ extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k
     }
     int* idx = idx_out ? idx_out + off * p->k : idx_ws;
     const long long hstride = idx_out ? T * p->k : (long long)n * p->k;
+    // attention over rows [a0, a1) as soon as their blocks are selected: one
+    // launch after all score chunks, or `parts` launches interleaved with them
+    int a0 = 0, part = 0;
     for (int q0 = 0; q0 < n; q0 += pl.chunk) {
       const int ql = n - q0 < pl.chunk ? n - q0 : pl.chunk;
+      if (hooks && (st = hooks->need_q(off + q0 + ql)) != INFV2_OK) return st;
       st = p->lse_approx
                ? launch_block_scores_approx(p, qs, kc1, kc2, n, q0, ql, s_shared, pl.ld, nullptr, cs)
                : launch_block_scores(p, qs, kc1, n, q0, ql, s_shared, pl.ld, nullptr, cs);
       if (st != INFV2_OK) return st;
       st = launch_select(p, s_shared, pl.ld, n, q0, ql, idx, hstride, cs);
       if (st != INFV2_OK) return st;
+      const int scored = q0 + ql;
+      if (scored == n || (parts > 1 && scored >= (long long)n * (part + 1) / parts)) {
+        st = launch_sparse_attn_rows(p, qs, ks, vs, idx, hstride, n, a0, scored, os, lses, T, cs);
+        if (st != INFV2_OK) return st;
+        if (hooks && (st = hooks->done_o(off + a0, off + scored)) != INFV2_OK) return st;
+        a0 = scored;
+        while (part < parts && scored >= (long long)n * (part + 1) / parts) ++part;
+      }
     }
-    st = launch_sparse_attn_prefill(p, qs, ks, vs, idx, hstride, n, os, lses, T, cs);
-    if (st != INFV2_OK) return st;
   }
   return INFV2_OK;
+}
+
+}  // namespace infv2
+
+extern "C" int infv2_prefill(const infv2_params* p, const void* q, const void* k, const void* v,
+                             const int* cu_seqlens_host, int batch, void* workspace,
+                             size_t ws_bytes, int* idx_out, void* o, float* lse,
+                             infv2_stream_t stream) {
+  return run_prefill(p, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                     static_cast<const uint16_t*>(v), cu_seqlens_host, batch, workspace, ws_bytes,
+                     idx_out, static_cast<uint16_t*>(o), lse, reinterpret_cast<cudaStream_t>(stream),
+                     nullptr);
 }
