@@ -515,8 +515,10 @@ def _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_over_ra
     every step copies its inputs from pinned host memory and reads its output
     back.  The library's pipeline copies on its own two streams into two
     device slots, so that step j+1's inputs travel and step j-1's output
-    returns while step j computes (as a serving loop would pipeline them);
-    every copy of every timed step is inside the timed region."""
+    returns while step j computes (as a serving loop would pipeline them), and
+    within a step the score chunks wait only for the Q rows they read and each
+    finished attention row range of O leaves while the next computes; every
+    copy of every timed step is inside the timed region."""
     qh = torch.from_numpy(data["q"].view(np.int16)).pin_memory()
     kh = torch.from_numpy(data["k"].view(np.int16)).pin_memory()
     vh = torch.from_numpy(data["v"].view(np.int16)).pin_memory()
@@ -545,8 +547,9 @@ def _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_over_ra
     return {"value": round(job_throughput(world, shape.n, ms), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "api": "infv2_pipeline_submit (host buffers)",
-            "overlap": "inputs of step j+1 and output of step j-1 copied on the pipeline's own "
-                       "streams while step j computes (two device slots)"}
+            "overlap": "Q copied in 8192-token parts and O returned per attention row range "
+                       "(8 per sequence) on the pipeline's own streams; step j+1's inputs and "
+                       "step j-1's output travel while step j computes (two device slots)"}
 
 
 def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, DecodeState):
