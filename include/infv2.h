@@ -262,7 +262,8 @@ int infv2_prefill(const infv2_params* p, const void* q, const void* k, const voi
  * Slot reuse is ordered by events, so any number of submits may be queued.
  * The library allocates no device memory for a pipeline: the caller's
  * workspace holds the prefill workspace and both slots.  The pipeline owns
- * two CUDA streams and its events, released by infv2_pipeline_destroy. */
+ * two CUDA streams and its events, released by infv2_pipeline_destroy.  A
+ * handle is not thread-safe: one host thread at a time may call into it. */
 typedef struct infv2_pipeline infv2_pipeline;
 
 /* Device workspace bytes a pipeline for this varlen batch needs: the
