@@ -553,8 +553,9 @@ def _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_over_ra
 
 
 def _decode(args, infv2, torch, shape3, rank, dev, stream, max_over_ranks, DecodeState):
-    """Batched decode: each step (append, K^C1 update, scores, selection,
-    split-KV attention, combine: 7 launches) is captured once into a CUDA graph,
+    """Batched decode: each step (3 launches: logits with the cache append and
+    K^C1 update; selection; split-KV attention whose last piece per row merges
+    and advances seqlens) is captured once into a CUDA graph,
     as a serving loop would run it, and the graphs are replayed in order (each
     replay appends its own token and advances seqlens on the device)."""
     cfg = dict(synth.CONFIGS["decode_batch32"])
