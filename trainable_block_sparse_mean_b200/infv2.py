@@ -342,7 +342,10 @@ def infv2_pipeline_workspace_size(p: Params, cu_seqlens) -> int:
 
 def infv2_pipeline_create(p: Params, cu_seqlens, workspace=None, stream=None,
                           device=None) -> Pipeline:
-    """Pipeline for prefill over host buffers; `stream` is the compute stream."""
+    """Pipeline for prefill over host buffers; `stream` is the compute stream.
+
+    The pipeline binds to the current CUDA device; `device` (where the
+    workspace is allocated when none is given) must be that device."""
     need = infv2_pipeline_workspace_size(p, cu_seqlens)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=device or "cuda")
