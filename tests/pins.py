@@ -528,4 +528,125 @@ def pin_attend_bwd_closed_forms():
     assert np.allclose(dk.sum(axis=0), 0.0, rtol=0, atol=1e-10), np.abs(dk.sum(axis=0)).max()
 
 
+# --------------------------------------------------------------------------
+# rounding, padding and the batch entry points
+# --------------------------------------------------------------------------
+
+_BF16_MAX = float(Fraction(2) ** 127 * (2 - Fraction(1, 128)))   # largest finite bf16
+
+
+def pin_compress_keeps_every_bf16_value():
+    """The mean of 32 copies of a bf16 value is that value, so compression must
+    return every finite bf16 bit pattern unchanged: every subnormal, 1.0, the
+    largest finite value.  A zero mean is +0 (the sum starts from +0, so 32
+    copies of -0 give +0: the sign of a zero is a convention, not a value)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = np.where((bits & 0x7F80) != 0x7F80, bits, 0).astype(np.uint16)
+    vals[vals == 0x8000] = 0
+    h_kv = 512
+    p = oracle.params(_shape(n=32, h_q=h_kv, h_kv=h_kv, d=128))
+    k = np.broadcast_to(vals.reshape(1, h_kv, 128), (32, h_kv, 128)).copy()
+    kc1 = oracle.compress_k(p, k)
+    assert kc1.shape == (1, h_kv, 128), kc1.shape
+    got = kc1[0].reshape(-1)
+    bad = np.nonzero(got != vals)[0]
+    assert bad.size == 0, [(hex(int(vals[x])), hex(int(got[x]))) for x in bad[:5]]
+
+
+def pin_bf16_round_nearest_even():
+    """Rounding of arbitrary doubles to bf16 against exact rational arithmetic:
+    normal and subnormal magnitudes, exact halfway points, and the overflow
+    edge (at or beyond the largest finite value plus half an ulp: infinity)."""
+    rng = np.random.default_rng(31)
+    xs = list(rng.standard_normal(300) * np.exp2(rng.integers(-140, 128, 300)))
+    for b in rng.integers(0, 0x7F7F, 200):             # midpoints between neighbours
+        lo = float(_f64(np.array([b], np.uint16))[0])
+        hi = float(_f64(np.array([b + 1], np.uint16))[0])
+        xs += [(lo + hi) / 2, -(lo + hi) / 2]
+    half_ulp = float(Fraction(2) ** (127 - 8))
+    xs += [_BF16_MAX, _BF16_MAX + half_ulp / 2, _BF16_MAX + half_ulp, 1.0, -1.0, 2.0 ** -133,
+           2.0 ** -134, 3 * 2.0 ** -135, 0.0, -0.0]
+    for x in xs:
+        got = float(_f64(np.array([oracle.bf16_round(x)], np.uint16))[0])
+        want = _rne_bf16_fraction(Fraction(x))
+        if abs(want) > _BF16_MAX:
+            want = np.copysign(np.inf, x)
+        assert got == want and np.signbit(got) == np.signbit(x if x != 0 else x), (x, got, want)
+
+
+def pin_batch_rows_match_single_rows():
+    """The batch entry points (several rows, two kv heads) put every row and
+    head where the single-row stages put it: S^shared (zero beyond the visible
+    kernels), the score log-sum-exp, S^cmp (minus infinity beyond the query's
+    block), the selection and the attention."""
+    for n in (700, 640):                               # 640: a whole number of blocks
+        _batch_rows_case(n, np.array([0, 40, 64, 300, 511, n - 60, n - 1], np.int32))
+
+
+def _batch_rows_case(n, rows):
+    sh, data = _small_problem(n=n, h_q=8, h_kv=2, d=16, seed=21, k=4)
+    p = oracle.params(sh)
+    G = sh.h_q // sh.h_kv
+    out = oracle.prefill_rows(p, data["q"], data["k"], data["v"], rows, want_cmp=True,
+                              want_shared=True, want_score_lse=True)
+    kc1 = oracle.compress_k(p, data["k"])
+    nc = oracle.num_kernels(p, sh.n)
+    for r, i in enumerate(rows):
+        nv = oracle.visible_kernels(p, int(i))
+        bi = int(i) // 64
+        for g in range(sh.h_kv):
+            s_row, lse = oracle.shared_scores_row(p, data["q"], kc1, int(i), g)
+            assert np.array_equal(out["shared"][r, g, :nv], s_row), (i, g)
+            assert np.all(out["shared"][r, g, nv:nc] == 0.0), (i, g)
+            assert np.array_equal(out["score_lse"][r, g * G:(g + 1) * G], lse), (i, g)
+            cmp_row = oracle.block_scores_row(p, s_row, int(i))
+            assert np.array_equal(out["cmp"][r, g, :bi + 1], cmp_row), (i, g)
+            assert np.all(out["cmp"][r, g, bi + 1:] == -np.inf), (i, g)
+            idx = oracle.select_row(p, cmp_row, int(i))
+            assert np.array_equal(out["idx"][r, g], idx), (i, g)
+            o, l = oracle.attend_row(p, data["q"], data["k"], data["v"], int(i), g, idx)
+            assert np.array_equal(out["o"][r, g * G:(g + 1) * G], o), (i, g)
+            assert np.array_equal(out["lse"][r, g * G:(g + 1) * G], l), (i, g)
+    # the selection and attention batch entries over the same rows
+    ld = nc + 5
+    shared = np.full((len(rows), sh.h_kv, ld), 7.0)    # padding beyond nv must not be read
+    for r, i in enumerate(rows):
+        nv = oracle.visible_kernels(p, int(i))
+        shared[r, :, :nv] = out["shared"][r, :, :nv]
+    n_blk = (sh.n + 63) // 64
+    idx, cmp_ = oracle.select_rows(p, shared, rows, n_blk)
+    assert np.array_equal(idx, out["idx"])
+    assert np.array_equal(cmp_, out["cmp"])
+    o, lse = oracle.attend_rows(p, data["q"], data["k"], data["v"], rows, out["idx"])
+    assert np.array_equal(o, out["o"]) and np.array_equal(lse, out["lse"])
+
+
+def pin_attend_empty_block_list():
+    """A query that selected no block attends to nothing: O = 0, lse = -inf."""
+    sh, data = _small_problem(n=200, h_q=4, h_kv=2, d=16, seed=3, k=4)
+    p = oracle.params(sh)
+    o, lse = oracle.attend_row(p, data["q"], data["k"], data["v"], 150, 1, [-1, -1, -1, -1])
+    assert np.all(o == 0.0) and np.all(lse == -np.inf), (o, lse)
+
+
+def pin_maxpool_literal_window():
+    """The literal reading of the max-pool window (kernels 4b .. 4b+4 of the
+    visible ones; pool_rule = 1), by brute force, and that it differs from
+    the intersection rule exactly where kernel 4b-1 or 4b+4 decides the max."""
+    p1 = oracle.params(_shape(), pool_rule=1)
+    p0 = oracle.params(_shape())
+    rng = np.random.default_rng(8)
+    differs = 0
+    for i in (31, 63, 64, 95, 130, 511, 700):
+        nv = oracle.visible_kernels(p1, i)
+        shared = rng.random(nv)
+        got = oracle.block_scores_row(p1, shared, i)
+        inter = oracle.block_scores_row(p0, shared, i)
+        for b in range(i // 64 + 1):
+            win = [shared[j] for j in range(4 * b, 4 * b + 5) if j < nv]
+            assert got[b] == (max(win) if win else -np.inf), (i, b)
+            differs += got[b] != inter[b]
+    assert differs > 0
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]
