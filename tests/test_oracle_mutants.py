@@ -53,6 +53,12 @@ MUTANTS = {
     "bwd_dk_unscaled": ("dk_acc[kv + c] += p->scale * ds * bf16_value(qr[c]);", "dk_acc[kv + c] += ds * bf16_value(qr[c]);"),
     "bwd_dv_from_ds": ("dv_acc[kv + c] += P[a] * bf16_value(dor[c]);", "dv_acc[kv + c] += ds * bf16_value(dor[c]);"),
     "kernel_window_short": ("t < j * p->s_c1 + p->l_c1; ++t", "t < j * p->s_c1 + p->l_c1 - 1; ++t"),
+    "bf16_overflow_edge": ("if (y > 3.3895313892515355e38) f = INFINITY;", "if (y >= 3.3895313892515355e38) f = INFINITY;"),
+    "empty_list_divides_by_zero": ("orow[c] = ntok ? orow[c] / L : 0.0;", "orow[c] = orow[c] / L;"),
+    "shared_padding_not_zero": ("so[j] = j < nv ? shared[j] : 0.0;", "so[j] = j < nv ? shared[j] : 1.0;"),
+    "cmp_drops_own_block": ("co[b] = b <= bi ? cmp[b] : -INFINITY;", "co[b] = b < bi ? cmp[b] : -INFINITY;"),
+    "blocks_floor_not_ceil": ("int n_blk = (n + p->B - 1) / p->B;\n    int G = p->h_q / p->h_kv;", "int n_blk = n / p->B + 1;\n    int G = p->h_q / p->h_kv;"),
+    "batch_row_stride_dropped": ("orc_select_row(p, cmp, i, idx_out + ((size_t)r * p->h_kv + g) * p->k);", "orc_select_row(p, cmp, i, idx_out + ((size_t)r + g) * p->k);"),
 }
 
 
