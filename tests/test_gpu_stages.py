@@ -61,6 +61,21 @@ def test_compress_extreme_values_bit_exact():
     assert np.array_equal(got, want)
 
 
+def test_compress_every_bf16_value_bit_exact():
+    # 32 equal rows per value: every finite bf16 bit pattern (subnormals, the
+    # largest finite value) is its own mean; a zero mean is +0 on both sides
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = np.where((bits & 0x7F80) != 0x7F80, bits, 0).astype(np.uint16)
+    sh = synth.Shape(n=32, h_q=512, h_kv=512)
+    kb = np.broadcast_to(vals.reshape(1, 512, 128), (32, 512, 128)).copy()
+    p = infv2.params_of(sh)
+    got = to_host_bits(infv2.infv2_compress_k(p, to_dev(kb)))
+    want = oracle.compress_k(oracle.params(sh), kb)
+    assert np.array_equal(got, want)
+    vals[vals == 0x8000] = 0
+    assert np.array_equal(got[0].reshape(-1), vals)
+
+
 # ---------------------------------------------------------------- stage 2
 
 SCORE_REL = 2e-5   # fp32 tensor-core dot products + fp32 softmax vs fp64
