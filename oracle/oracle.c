@@ -24,7 +24,8 @@
  * Readings where the pages are silent (each also listed in the design notes):
  *  - scale 1/sqrt(d) on the score logits and the attention logits (parameter);
  *  - a kernel is visible to query i only when its last token is <= i;
- *  - K^C1 is a bf16 tensor: the exact mean rounded once, nearest-even;
+ *  - K^C1 is a bf16 tensor: the exact mean rounded once, nearest-even (the
+ *    fp64 sum starts at +0, so a zero mean is +0);
  *  - the local set is {b_i - n_local + 1 .. b_i} (own block included);
  *  - k counts every selected block, init and local included;
  *  - equal block scores are ordered by lower block index;
@@ -37,6 +38,11 @@
  *    over the visible coarse kernels plus log(s_C2 / s_C1) (each coarse kernel
  *    stands for that many stage-1 kernels), and a row that sees no coarse
  *    kernel keeps the exact log-sum-exp.
+ *
+ * Parity unpinned: two readings that no page fixes with a worked example,
+ * the choice of the intersection rule over the literal max-pool window
+ * (both are built; pool_rule selects) and the 1/sqrt(d) logit scale.  Every
+ * function is pinned under those readings by the tests' pins.
  */
 #include <math.h>
 #include <stdint.h>
