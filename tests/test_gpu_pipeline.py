@@ -108,3 +108,24 @@ def test_pipeline_join_orders_a_stream_after_the_copies():
     torch.cuda.synchronize()
     assert np.array_equal(o.numpy().view(np.uint16), _bits(want))
     infv2.infv2_pipeline_destroy(pl)
+
+
+@pytest.mark.parametrize("lengths", [[0, 300, 0, 1000], [300, 400]])
+def test_pipeline_empty_and_dense_only_batches(lengths):
+    # empty sequences between the others; an all-dense batch (no prefill workspace)
+    sh = synth.Shape(n=0, h_q=8, h_kv=2, k=8)
+    d = synth.make_varlen(sh, lengths, seed=4)
+    cu = [int(x) for x in d["cu_seqlens"]]
+    T = cu[-1]
+    p = infv2.params_of(sh)
+    pl = infv2.infv2_pipeline_create(p, cu)
+    o = torch.zeros((T, sh.h_q, sh.d), dtype=torch.int16).pin_memory()
+    lse = torch.zeros((sh.h_q, T)).pin_memory()
+    infv2.infv2_pipeline_submit(pl, _pinned(d["q"]), _pinned(d["k"]), _pinned(d["v"]), o, lse)
+    infv2.infv2_pipeline_sync(pl)
+    infv2.infv2_pipeline_destroy(pl)
+    want_lse = torch.empty((sh.h_q, T), device="cuda")
+    want = infv2.infv2_prefill(p, to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"]), cu, lse=want_lse)
+    torch.cuda.synchronize()
+    assert np.array_equal(o.numpy().view(np.uint16), _bits(want))
+    assert torch.equal(lse, want_lse.cpu())
