@@ -92,6 +92,32 @@ def max_over_ranks(dist, x: float, device) -> float:
     return float(t.item())
 
 
+def needle_recall(sel, needles, B: int = 64, span: int = 32):
+    """Sanity figure of the synthetic needles (not parity): the share of
+    (needle, kv head) pairs whose target query selected a block that the
+    needle's span of `span` keys intersects.  sel: [h_kv, len(needles), k]
+    block lists at the needles' target rows; needles: (target, span start)."""
+    found = total = 0
+    for r, (_, p0) in enumerate(needles):
+        blocks = {p0 // B, (p0 + span - 1) // B}
+        for g in range(sel.shape[0]):
+            total += 1
+            found += bool(blocks & {int(x) for x in sel[g, r]})
+    return {"found": found, "total": total, "recall": round(found / total, 4) if total else None}
+
+
+def _needle_recall_of(idx, needles):
+    """needle_recall on the benchmark's own block lists [h_kv, n, k] (device)."""
+    try:
+        if idx is None or not needles:
+            return None
+        import torch
+        rows = torch.tensor([t for t, _ in needles], dtype=torch.long, device=idx.device)
+        return needle_recall(idx.index_select(1, rows).cpu().numpy(), needles)
+    except Exception as e:   # a sanity figure never ends the benchmark
+        return {"error": str(e)[:200]}
+
+
 def job_throughput(world: int, units_per_rank: int, ms_per_step: float) -> float:
     """Whole-job units/s: every rank processes its own replica; the step time
     is the slowest rank's."""
@@ -318,6 +344,7 @@ def run_ours(args, rank, world, local_rank, dist):
         "lse_approx": approx,
         "backward": bwd,
         "roofline": roof,
+        "needle_recall": _needle_recall_of(stage.get("idx"), data.get("needles")),
         "e2e": e2e,
         "decode": dec,
         "gpu_launches": launches_per_step * args.steps,
@@ -399,7 +426,7 @@ def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, 
     per["select_kernel"]["bytes_per_step"] = float(p.h_kv * vis * 4 + p.h_kv * n * p.k * 4)
     for nm in names:
         per[nm] = {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in per[nm].items()}
-    return dict(per_kernel=per, ms_per_step=e0.elapsed_time(e1) / steps)
+    return dict(per_kernel=per, ms_per_step=e0.elapsed_time(e1) / steps, idx=idx)
 
 
 def _fused_pool_timing(args, infv2, torch, p, shape, q, k, ws, stream, chunk_rows, stage):

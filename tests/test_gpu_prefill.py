@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 import torch
 
+import bench
 import oracle
 import parity
 from trainable_block_sparse_mean_b200 import build as build_mod
@@ -97,6 +98,10 @@ def test_prefill_32k_sampled():
     rows = _rows(sh.n, 120, 2)
     rows = np.unique(np.concatenate([rows, [t for t, _ in data["needles"]]])).astype(np.int32)
     check_sequence(sh, data, dev, 0, sh.n, rows, dense=False)
+    # sanity figure: every planted needle's block is selected by its target query
+    targets = torch.tensor([t for t, _ in data["needles"]], dtype=torch.long, device="cuda")
+    sel = dev["idx"].index_select(1, targets).cpu().numpy()
+    assert bench.needle_recall(sel, data["needles"])["recall"] == 1.0
 
 
 @pytest.mark.slow
