@@ -39,10 +39,11 @@
  *    stands for that many stage-1 kernels), and a row that sees no coarse
  *    kernel keeps the exact log-sum-exp.
  *
- * Parity unpinned: two readings that no page fixes with a worked example,
- * the choice of the intersection rule over the literal max-pool window
- * (both are built; pool_rule selects) and the 1/sqrt(d) logit scale.  Every
- * function is pinned under those readings by the tests' pins.
+ * Parity unpinned: readings that no page fixes with a worked example, namely
+ * the choice of the intersection rule over the literal max-pool window (both
+ * are built; pool_rule selects), the 1/sqrt(d) logit scale, and in the
+ * optional LSE approximation the bf16 rounding of K^C2 and the log(s_C2/s_C1)
+ * constant.  Every function is pinned under those readings by the tests' pins.
  */
 #include <math.h>
 #include <stdint.h>
