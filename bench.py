@@ -92,6 +92,33 @@ def max_over_ranks(dist, x: float, device) -> float:
     return float(t.item())
 
 
+MUFU_PER_SM_CLK = 16   # ex2 per SM per clock (CUDA programming guide, arithmetic throughput)
+FMA_EXP_SHARE = 0.25   # share of the score kernel's exponentials on the FMA-pipe polynomial
+
+
+def score_exp_figures(n: int, h_q: int, ms_score: float, sms: int, sm_mhz: float):
+    """The score kernel's secondary bound: one exponential per (head, visible
+    kernel) in each of its two passes, against the MUFU rate at the clock the
+    run saw.  mufu_frac counts the share that the MUFU executes."""
+    exps = 2.0 * h_q * float(visible_kernels(np.arange(n)).sum())
+    rate = exps / (ms_score / 1e3)
+    peak = MUFU_PER_SM_CLK * sms * sm_mhz * 1e6
+    return {"exp_per_step": exps, "exp_per_s": round(rate, 1), "mufu_peak_per_s": round(peak, 1),
+            "sm_count": sms, "sm_mhz": sm_mhz, "fma_share": FMA_EXP_SHARE,
+            "mufu_frac": round(rate * (1.0 - FMA_EXP_SHARE) / peak, 4)}
+
+
+def _score_exp_of(n, h_q, stage, dev, clk):
+    try:
+        import torch
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = float(clk["sm_mhz"]) if clk and clk.get("sm_mhz") else 1965.0
+        ms = stage["per_kernel"]["score_kernel"]["ms_per_step"]
+        return score_exp_figures(n, h_q, ms, sms, mhz)
+    except Exception as e:   # a secondary figure never ends the benchmark
+        return {"error": str(e)[:200]}
+
+
 def needle_recall(sel, needles, B: int = 64, span: int = 32):
     """Sanity figure of the synthetic needles (not parity): the share of
     (needle, kv head) pairs whose target query selected a block that the
@@ -345,6 +372,7 @@ def run_ours(args, rank, world, local_rank, dist):
         "backward": bwd,
         "roofline": roof,
         "needle_recall": _needle_recall_of(stage.get("idx"), data.get("needles")),
+        "score_exp": _score_exp_of(n, p.h_q, stage, dev, clk),
         "e2e": e2e,
         "decode": dec,
         "gpu_launches": launches_per_step * args.steps,

@@ -1,6 +1,7 @@
 """The synthetic needles as a sanity figure (not parity): the benchmark's
 needle_recall counting rule on a hand example, and the oracle's selection
-finding every planted needle on a small needle workload."""
+finding every planted needle on a small needle workload; the closed form of
+the score kernel's exponential count."""
 import numpy as np
 
 import bench
@@ -30,3 +31,17 @@ def test_oracle_finds_every_planted_needle():
     out = oracle.prefill_rows(oracle.params(sh), data["q"], data["k"], data["v"], rows)
     rec = bench.needle_recall(out["idx"].transpose(1, 0, 2), data["needles"])
     assert rec["recall"] == 1.0, rec
+
+
+def test_score_exp_figures_closed_form():
+    # one exponential per (head, visible kernel) in each pass; kernel j is
+    # visible to query i when 16j + 31 <= i
+    n, h_q = 4100, 8
+    vis = sum((i - 31) // 16 + 1 for i in range(31, n))
+    f = bench.score_exp_figures(n, h_q, 2.0, 148, 1965.0)
+    assert f["exp_per_step"] == 2 * h_q * vis
+    assert abs(f["exp_per_s"] - 2 * h_q * vis / 2e-3) < 1.0
+    assert f["mufu_peak_per_s"] == 16 * 148 * 1965e6
+    assert abs(f["mufu_frac"] - 0.75 * f["exp_per_s"] / f["mufu_peak_per_s"]) < 1e-4
+    big = bench.score_exp_figures(131072, 32, 1.0, 148, 1965.0)["exp_per_step"]
+    assert abs(big - 3.43e10) / 3.43e10 < 0.01
