@@ -198,6 +198,18 @@ int infv2_select_topk_pooled(const infv2_params* p, const float* s_cmp, int ld_c
 int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const void* v,
                       const int* idx, int n, void* o, float* lse, infv2_stream_t stream);
 
+/* Stage 5 over query rows r0 .. r1-1 only (chunked prefill: the rows whose
+ * blocks have been selected so far).  Tensors are the whole sequence's, as in
+ * infv2_sparse_attn; rows outside [r0, r1) of o and lse are not written and
+ * rows of idx outside it are not read.  idx NULL: dense causal attention
+ * (every block up to the query's own).  Only K/V rows below the last block
+ * boundary at or after r1 are read.  0 <= r0 <= r1 <= n, else
+ * INFV2_ERR_INVALID_ARG; r0 == r1 does nothing.  The results of any split of
+ * [0, n) into ranges equal infv2_sparse_attn's bit for bit. */
+int infv2_sparse_attn_rows(const infv2_params* p, const void* q, const void* k, const void* v,
+                           const int* idx, int n, int r0, int r1, void* o, float* lse,
+                           infv2_stream_t stream);
+
 /* Workspace bytes that infv2_sparse_attn_bwd needs for an n-token sequence
  * (either mode: block lists or dense). */
 int infv2_sparse_attn_bwd_workspace_size(const infv2_params* p, int n, size_t* bytes);

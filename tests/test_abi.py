@@ -107,6 +107,12 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_select_topk_pooled(P, 16, 2, 100, 0, 10, 16, None) == infv2.ERR_INVALID_ARG
     assert L.infv2_select_topk_pooled(P, 8, 4, 100, 0, 10, 16, None) == infv2.ERR_INVALID_ARG  # misaligned
     assert L.infv2_sparse_attn(P, None, None, None, None, 10, None, None, None) == infv2.ERR_INVALID_ARG
+    # row ranges: bounds checked first; an empty range does nothing
+    assert L.infv2_sparse_attn_rows(P, None, None, None, None, 100, 5, 5, None, None, None) == infv2.OK
+    assert L.infv2_sparse_attn_rows(P, None, None, None, None, 100, 0, 10, None, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_sparse_attn_rows(P, 16, 16, 16, None, 100, -1, 10, 16, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_sparse_attn_rows(P, 16, 16, 16, None, 100, 20, 10, 16, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_sparse_attn_rows(P, 16, 16, 16, None, 100, 0, 101, 16, None, None) == infv2.ERR_INVALID_ARG
     assert L.infv2_dense_attn(P, None, None, None, 0, None, None, None) == infv2.OK
     assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,
                           None, None) == infv2.OK

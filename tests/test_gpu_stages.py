@@ -300,6 +300,36 @@ def test_dense_attn_matches_oracle(n, h_q, h_kv):
     assert np.allclose(lse.cpu().numpy()[:, rows].T, ref["lse"], rtol=0, atol=2e-3)
 
 
+@pytest.mark.parametrize("dense", [False, True])
+def test_attn_rows_split_equals_whole(dense):
+    """Chunked prefill: attention over row ranges (the oracle's block lists, or
+    dense) equals the whole-sequence call bit for bit; rows outside a range
+    are left alone."""
+    n, h_q, h_kv, k = 3000, 16, 2, 8
+    sh, d = _problem(n, h_q, h_kv, k=k, seed=29)
+    p = infv2.params_of(sh)
+    q, kk, vv = to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"])
+    ii = None
+    if not dense:
+        ref = oracle.prefill_rows(oracle.params(sh), d["q"], d["k"], d["v"], np.arange(n, dtype=np.int32))
+        ii = torch.from_numpy(ref["idx"].transpose(1, 0, 2).copy()).cuda()
+    lse = torch.empty((h_q, n), device="cuda")
+    whole = (infv2.infv2_dense_attn(p, q, kk, vv, lse=lse) if dense
+             else infv2.infv2_sparse_attn(p, q, kk, vv, ii, lse=lse))
+    o = torch.full_like(q, 7.0)
+    lse2 = torch.full((h_q, n), 7.0, device="cuda")
+    cuts = [0, 1, 64, 700, 701, 2048, 2999, 3000]
+    for r0, r1 in zip(cuts[:-1], cuts[1:]):
+        infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, r0, r1, o=o, lse=lse2)
+        torch.cuda.synchronize()
+        assert torch.all(o[r1:].view(torch.int16) == torch.full_like(q, 7.0)[r1:].view(torch.int16))
+    infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, 5, 5, o=o, lse=lse2)   # empty: no-op
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    assert torch.equal(o.view(torch.int16), whole.view(torch.int16))
+    assert torch.equal(lse2, lse)
+
+
 def test_timeout_path_reports_and_recovers():
     assert infv2.infv2_device_status() == 0
     infv2.infv2_selftest_timeout(2000)

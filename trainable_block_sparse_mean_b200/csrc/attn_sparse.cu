@@ -594,6 +594,20 @@ extern "C" int infv2_sparse_attn(const infv2_params* p, const void* q, const voi
                                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" int infv2_sparse_attn_rows(const infv2_params* p, const void* q, const void* k,
+                                      const void* v, const int* idx, int n, int r0, int r1,
+                                      void* o, float* lse, infv2_stream_t stream) {
+  int st = infv2_check_params(p);
+  if (st != INFV2_OK) return st;
+  if (n < 0 || r0 < 0 || r1 > n || r0 > r1) return INFV2_ERR_INVALID_ARG;
+  if (r0 == r1) return INFV2_OK;
+  if (!q || !k || !v || !o) return INFV2_ERR_INVALID_ARG;
+  return launch_sparse_attn_rows(p, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                 static_cast<const uint16_t*>(v), idx, idx ? (long long)n * p->k : 0,
+                                 n, r0, r1, static_cast<uint16_t*>(o), lse, n,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 namespace infv2 {
 // Dense causal attention through the same kernel with every visible block.
 int launch_dense_attn_blocks(const infv2_params* p, const uint16_t* q, const uint16_t* k,

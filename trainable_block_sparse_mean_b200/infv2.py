@@ -26,7 +26,7 @@ SYMBOLS = [
     "infv2_compress_k2", "infv2_block_scores_approx", "infv2_sparse_attn_bwd_workspace_size",
     "infv2_sparse_attn_bwd", "infv2_pipeline_workspace_size", "infv2_pipeline_create",
     "infv2_pipeline_submit", "infv2_pipeline_wait", "infv2_pipeline_join", "infv2_pipeline_sync",
-    "infv2_pipeline_destroy",
+    "infv2_pipeline_destroy", "infv2_sparse_attn_rows",
 ]
 
 
@@ -73,6 +73,7 @@ def lib():
         L.infv2_block_scores_approx.argtypes = [P, vp, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk_pooled.argtypes = [P, vp, i, i, i, i, vp, vp]
         L.infv2_sparse_attn.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
+        L.infv2_sparse_attn_rows.argtypes = [P, vp, vp, vp, vp, i, i, i, vp, vp, vp]
         L.infv2_dense_attn.argtypes = [P, vp, vp, vp, i, vp, vp, vp]
         L.infv2_prefill_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
         L.infv2_prefill.argtypes = [P, vp, vp, vp, vp, i, vp, sz, vp, vp, vp, vp]
@@ -243,6 +244,18 @@ def infv2_sparse_attn(p: Params, q, k, v, idx, o=None, lse=None, stream=None):
         o = torch.empty_like(q)
     _check(lib().infv2_sparse_attn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), n,
                                    _ptr(o), _ptr(lse), _stream(stream)), "infv2_sparse_attn")
+    return o
+
+
+def infv2_sparse_attn_rows(p: Params, q, k, v, idx, r0: int, r1: int, o=None, lse=None,
+                           stream=None):
+    """Attention over query rows r0..r1-1 of the sequence (idx None: dense)."""
+    n = q.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_sparse_attn_rows(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), n,
+                                        r0, r1, _ptr(o), _ptr(lse), _stream(stream)),
+           "infv2_sparse_attn_rows")
     return o
 
 
