@@ -198,8 +198,9 @@ int infv2_select_topk_pooled(const infv2_params* p, const float* s_cmp, int ld_c
 int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const void* v,
                       const int* idx, int n, void* o, float* lse, infv2_stream_t stream);
 
-/* Stage 5 over query rows r0 .. r1-1 only (chunked prefill: the rows whose
- * blocks have been selected so far).  Tensors are the whole sequence's, as in
+/* Stage 5 over query rows r0 .. r1-1 only (a prefill computed in row chunks:
+ * the rows whose blocks have been selected so far).  Tensors are the whole
+ * sequence's, as in
  * infv2_sparse_attn; rows outside [r0, r1) of o and lse are not written and
  * rows of idx outside it are not read.  idx NULL: dense causal attention
  * (every block up to the query's own).  Only K/V rows below the last block
