@@ -200,11 +200,10 @@ int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const
 
 /* Stage 5 over query rows r0 .. r1-1 only (a prefill computed in row chunks:
  * the rows whose blocks have been selected so far).  Tensors are the whole
- * sequence's, as in
- * infv2_sparse_attn; rows outside [r0, r1) of o and lse are not written and
- * rows of idx outside it are not read.  idx NULL: dense causal attention
- * (every block up to the query's own).  Only K/V rows below the last block
- * boundary at or after r1 are read.  0 <= r0 <= r1 <= n, else
+ * sequence's, as in infv2_sparse_attn; rows outside [r0, r1) of o and lse
+ * are not written and rows of idx outside it are not read.  idx NULL: dense
+ * causal attention (every block up to the query's own).  Only K/V rows below
+ * the last block boundary at or after r1 are read.  0 <= r0 <= r1 <= n, else
  * INFV2_ERR_INVALID_ARG; r0 == r1 does nothing.  The results of any split of
  * [0, n) into ranges equal infv2_sparse_attn's bit for bit. */
 int infv2_sparse_attn_rows(const infv2_params* p, const void* q, const void* k, const void* v,
