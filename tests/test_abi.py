@@ -181,3 +181,14 @@ def test_pipeline_binding_checks_host_buffer_sizes():
     with pytest.raises(ValueError):
         infv2.infv2_pipeline_submit(pl, q, torch.zeros((100, 2, 128), dtype=torch.bfloat16)[:, :1], kv, q)
     infv2.infv2_pipeline_destroy(pl)   # a handle that was never created: no-op
+
+
+def test_binding_refuses_host_tensors():
+    # device-pointer entry points take CUDA tensors only: a CPU tensor never
+    # reaches the library, so there is no silent host path
+    import torch
+    p = infv2.params(4, 1)
+    q = torch.zeros((64, 4, 128), dtype=torch.bfloat16)
+    kv = torch.zeros((64, 1, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        infv2.infv2_dense_attn(p, q, kv, kv, o=q)
