@@ -204,8 +204,12 @@ int infv2_sparse_attn(const infv2_params* p, const void* q, const void* k, const
  * are not written and rows of idx outside it are not read.  idx NULL: dense
  * causal attention (every block up to the query's own).  Only K/V rows below
  * the last block boundary at or after r1 are read.  0 <= r0 <= r1 <= n, else
- * INFV2_ERR_INVALID_ARG; r0 == r1 does nothing.  The results of any split of
- * [0, n) into ranges equal infv2_sparse_attn's bit for bit. */
+ * INFV2_ERR_INVALID_ARG; r0 == r1 does nothing.  A split of [0, n) into
+ * ranges whose ends are multiples of 128/G tokens (the attention's query tile;
+ * G = h_q / h_kv) or n gives infv2_sparse_attn's results bit for bit; ends
+ * inside a tile give results equal to within rounding (a row's probabilities
+ * are rounded against a reference maximum that the other tokens of its tile
+ * can move). */
 int infv2_sparse_attn_rows(const infv2_params* p, const void* q, const void* k, const void* v,
                            const int* idx, int n, int r0, int r1, void* o, float* lse,
                            infv2_stream_t stream);

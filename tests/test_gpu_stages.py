@@ -303,9 +303,13 @@ def test_dense_attn_matches_oracle(n, h_q, h_kv):
 @pytest.mark.parametrize("dense", [False, True])
 def test_attn_rows_split_equals_whole(dense):
     """Chunked prefill: attention over row ranges (the oracle's block lists, or
-    dense) equals the whole-sequence call bit for bit; rows outside a range
-    are left alone."""
+    dense) leaves rows outside a range alone; ranges that end on tile
+    boundaries (multiples of 128/G tokens) give the whole-sequence call's bits,
+    and ranges that cut a tile agree with it to within rounding (a row's
+    probabilities are rounded against a reference maximum that the other
+    tokens of its tile can move)."""
     n, h_q, h_kv, k = 3000, 16, 2, 8
+    tq = 128 // (h_q // h_kv)
     sh, d = _problem(n, h_q, h_kv, k=k, seed=29)
     p = infv2.params_of(sh)
     q, kk, vv = to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"])
@@ -316,18 +320,24 @@ def test_attn_rows_split_equals_whole(dense):
     lse = torch.empty((h_q, n), device="cuda")
     whole = (infv2.infv2_dense_attn(p, q, kk, vv, lse=lse) if dense
              else infv2.infv2_sparse_attn(p, q, kk, vv, ii, lse=lse))
-    o = torch.full_like(q, 7.0)
-    lse2 = torch.full((h_q, n), 7.0, device="cuda")
-    cuts = [0, 1, 64, 700, 701, 2048, 2999, 3000]
-    for r0, r1 in zip(cuts[:-1], cuts[1:]):
-        infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, r0, r1, o=o, lse=lse2)
+    for cuts, exact in (([0, tq, 64, 44 * tq, 2048, n - n % tq, n], True),
+                        ([0, 1, 64, 700, 701, 2048, 2999, n], False)):
+        o = torch.full_like(q, 7.0)
+        lse2 = torch.full((h_q, n), 7.0, device="cuda")
+        for r0, r1 in zip(cuts[:-1], cuts[1:]):
+            infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, r0, r1, o=o, lse=lse2)
+            torch.cuda.synchronize()
+            assert torch.all(o[r1:].view(torch.int16) == torch.full_like(q, 7.0)[r1:].view(torch.int16))
+        infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, 5, 5, o=o, lse=lse2)   # empty: no-op
         torch.cuda.synchronize()
-        assert torch.all(o[r1:].view(torch.int16) == torch.full_like(q, 7.0)[r1:].view(torch.int16))
-    infv2.infv2_sparse_attn_rows(p, q, kk, vv, ii, 5, 5, o=o, lse=lse2)   # empty: no-op
-    torch.cuda.synchronize()
-    assert infv2.infv2_device_status() == 0
-    assert torch.equal(o.view(torch.int16), whole.view(torch.int16))
-    assert torch.equal(lse2, lse)
+        assert infv2.infv2_device_status() == 0
+        if exact:
+            assert torch.equal(o.view(torch.int16), whole.view(torch.int16))
+            assert torch.equal(lse2, lse)
+        else:
+            parity.assert_outputs_close(o.float().cpu().numpy(), whole.double().cpu().numpy(),
+                                        "row ranges cutting tiles")
+            assert float((lse2 - lse).abs().max()) <= 1e-3
 
 
 def test_timeout_path_reports_and_recovers():

@@ -543,6 +543,9 @@ int launch_sparse_attn_rows(const infv2_params* p, const uint16_t* q, const uint
                             cudaStream_t st) {
   if (r0 < 0 || r1 > n || r0 > r1) return INFV2_ERR_INVALID_ARG;
   if (r1 == r0) return INFV2_OK;
+  // tiles of 128 (token, head) rows on the tensor cores wherever the shape allows
+  if (attn_tc_supports(p, idx == nullptr))
+    return launch_attn_tc(p, q, k, v, idx, idx_hstride, n, r0, r1, o, lse, lse_ld, st);
   CUtensorMap tm_k, tm_v;
   if (!make_tmap_3d(&tm_k, k, 128, p->h_kv, n, 256, (uint64_t)p->h_kv * 256, 64, 1, 64) ||
       !make_tmap_3d(&tm_v, v, 128, p->h_kv, n, 256, (uint64_t)p->h_kv * 256, 64, 1, 64))

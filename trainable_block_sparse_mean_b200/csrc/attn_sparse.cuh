@@ -46,6 +46,20 @@ int launch_sparse_attn_rows(const infv2_params* p, const uint16_t* q, const uint
 }  // namespace infv2
 
 namespace infv2 {
+// Block-list entries (tokens per tile x k) that one tile of the tensor-core
+// attention can stage: sparse lists need G >= 4 and (128/G)*k <= this.
+constexpr int kTcListCap = 2048;
+
+// Whether the tensor-core attention takes this shape (dense: every G).
+bool attn_tc_supports(const infv2_params* p, bool dense);
+
+// Tensor-core attention over query rows [r0, r1) of an n-token sequence:
+// idx [h_kv][n][k] block lists (row stride k, kv-head stride idx_hstride), or
+// null for dense causal attention.
+int launch_attn_tc(const infv2_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const int* idx, long long idx_hstride, int n, int r0, int r1, uint16_t* o,
+                   float* lse, long long lse_ld, cudaStream_t st);
+
 int launch_dense_attn_blocks(const infv2_params* p, const uint16_t* q, const uint16_t* k,
                              const uint16_t* v, int n, uint16_t* o, float* lse, long long lse_ld,
                              cudaStream_t st);
