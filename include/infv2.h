@@ -355,6 +355,27 @@ int infv2_decode(const infv2_params* p, const void* q, const void* k_new, const 
                  void* workspace, size_t ws_bytes, int* idx_out, void* o, float* lse,
                  infv2_stream_t stream);
 
+/* The attention stage of infv2_decode alone, over block lists the caller
+ * gives (MiniCPM4 blog, query/key granularity: each decode query attends to
+ * its own blocks; arXiv summary, Appendix A: the kernel returns O and the
+ * log-sum-exp).  For sequence s, the query q[s] at position pos[s] attends to
+ * the cached tokens t <= pos[s] of the blocks in idx[s, g, :] (entries < 0
+ * ignored), with the split-KV kernel of the decode step.  Neither the caches
+ * nor pos are written: a caller can re-run the attention on a selection it
+ * holds (a verification, or a selection made elsewhere).
+ *   q        bf16 [batch, h_q, d]
+ *   k_cache, v_cache  bf16 [batch, h_kv, cap, d]
+ *   pos      int32 [batch] (device): 0 <= pos[s] < cap
+ *   idx      int32 [batch, h_kv, k]
+ *   workspace: >= infv2_decode_workspace_size(p, batch, cap) bytes, 256-byte
+ *            aligned (it may be the decode step's; calls that share it must be
+ *            ordered on the caller's streams)
+ *   o        bf16 [batch, h_q, d];  lse fp32 [batch, h_q] (nullable) */
+int infv2_decode_attn(const infv2_params* p, const void* q, const void* k_cache,
+                      const void* v_cache, const int* pos, int batch, int cap, const int* idx,
+                      void* workspace, size_t ws_bytes, void* o, float* lse,
+                      infv2_stream_t stream);
+
 /* Block selection (the work of infv2_block_scores followed by
  * infv2_select_topk) for callers that cannot allocate device memory: code that
  * runs inside a memory arena or pool it does not own, an engine whose

@@ -117,6 +117,14 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,
                           None, None) == infv2.OK
     assert L.infv2_selftest_timeout(0, None) == infv2.ERR_INVALID_ARG
+    # decode attention alone: an empty batch does nothing; bad shapes, missing
+    # pointers and a small or misaligned workspace are refused before any launch
+    assert L.infv2_decode_attn(P, None, None, None, None, 0, 16, None, None, 0, None, None, None) == infv2.OK
+    assert L.infv2_decode_attn(P, None, None, None, None, -1, 16, None, None, 0, None, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_decode_attn(P, 16, 16, 16, 16, 2, 0, 16, 256, 1 << 20, 16, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_decode_attn(P, 16, 16, 16, None, 2, 256, 16, 256, 1 << 20, 16, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_decode_attn(P, 16, 16, 16, 16, 2, 256, 16, 256, 64, 16, None, None) == infv2.ERR_WORKSPACE
+    assert L.infv2_decode_attn(P, 16, 16, 16, 16, 2, 256, 16, 16, 1 << 30, 16, None, None) == infv2.ERR_INVALID_ARG
     # the LSE approximation flag: 0 or 1; decode does not take it
     assert p.lse_approx == 0
     pa = infv2.params(32, 2, lse_approx=1)

@@ -1,7 +1,10 @@
 """Decode-step parity (infv2_decode through the C ABI): the appended cache
 rows, the incremental K^C1 (bit-exact against the oracle's compression of the
 same tokens), the selected blocks and the output of the query at position L,
-which must equal the oracle's prefill row L of the (L+1)-token sequence."""
+which must equal the oracle's prefill row L of the (L+1)-token sequence.  The
+decode attention is also re-run on the oracle's own block lists
+(infv2_decode_attn) for every checked row, so a row whose selection differs by
+a legal swap still has its output checked."""
 import numpy as np
 import pytest
 import torch
@@ -39,7 +42,7 @@ def run_and_check(shape, data, steps, check_seqs, check_steps):
     st = DecodeState(shape, data)
     op = oracle.params(shape)
     B = st.batch
-    stats = dict(equal=0, swapped=0)
+    stats = dict(equal=0, swapped=0, attn_checked=0)
     for t in range(steps):
         idx = torch.full((B, shape.h_kv, shape.k), -3, dtype=torch.int32, device="cuda")
         lse = torch.empty((B, shape.h_q), device="cuda")
@@ -52,6 +55,7 @@ def run_and_check(shape, data, steps, check_seqs, check_steps):
             continue
         og = synth.bf16_to_f32(to_host_bits(o))
         gi = idx.cpu().numpy()
+        refs = {}
         for s in check_seqs:
             L = int(data["lens"][s]) + t          # query position of this step
             k, v = _sequence_tokens(data, s, L + 1)
@@ -65,6 +69,23 @@ def run_and_check(shape, data, steps, check_seqs, check_steps):
             if n_sw == 0:
                 parity.assert_outputs_close(og[s:s + 1], ref["o"], f"decode seq {s} step {t}")
                 assert np.allclose(lse.cpu().numpy()[s], ref["lse"][0], atol=2e-3, rtol=0)
+            refs[s] = ref
+        # the decode attention on the oracle's block lists, for every checked row
+        idx_ref = idx.clone()
+        for s in check_seqs:
+            idx_ref[s] = torch.from_numpy(refs[s]["idx"][0]).cuda()
+        pos = torch.from_numpy((data["lens"] + t).astype(np.int32)).cuda()
+        lse2 = torch.empty((B, shape.h_q), device="cuda")
+        o2 = infv2.infv2_decode_attn(st.p, st.q[t], st.k_cache, st.v_cache, pos, idx_ref,
+                                     st.workspace, lse=lse2)
+        torch.cuda.synchronize()
+        assert infv2.infv2_device_status() == 0
+        assert torch.equal(pos.cpu(), torch.from_numpy((data["lens"] + t).astype(np.int32)))
+        og2 = synth.bf16_to_f32(to_host_bits(o2))
+        for s in check_seqs:
+            parity.assert_outputs_close(og2[s:s + 1], refs[s]["o"], f"decode attention seq {s} step {t}")
+            assert np.allclose(lse2.cpu().numpy()[s], refs[s]["lse"][0], atol=2e-3, rtol=0)
+            stats["attn_checked"] += 1
     # caches: appended rows and K^C1 of every complete kernel
     kc = to_host_bits(st.k_cache)
     vc = to_host_bits(st.v_cache)
@@ -110,12 +131,19 @@ def _with_lengths(sh, lens, steps, cap, seed):
 
 @pytest.mark.slow
 def test_decode_batch32_sampled():
+    """The batch-32 decode workload as configured: every sequence holds its own
+    seeded data (cache lengths U[16k, 128k]); eight sequences, the shortest and
+    the longest cache among them, are checked against the oracle on three
+    consecutive steps."""
     cfg = synth.CONFIGS["decode_batch32"]
     sh = cfg["shape"]
-    sample = [0, 7, 19, 31]
-    data = synth.make_decode(sh, cfg["batch"], cfg["len_lo"], cfg["len_hi"], 3, seed=0, only=sample)
-    stats = run_and_check(sh, data, 3, sample, check_steps={0, 2})
-    assert stats["equal"] + stats["swapped"] >= 2 * len(sample) * sh.h_kv
+    data = synth.make_decode(sh, cfg["batch"], cfg["len_lo"], cfg["len_hi"], 3, seed=0)
+    order = np.argsort(data["lens"])
+    sample = sorted({int(order[0]), int(order[-1]), 0, 7, 12, 19, 25, 31})
+    assert len(sample) >= 8
+    stats = run_and_check(sh, data, 3, sample, check_steps={0, 1, 2})
+    assert stats["equal"] + stats["swapped"] == 3 * len(sample) * sh.h_kv
+    assert stats["attn_checked"] == 3 * len(sample)
 
 
 def test_decode_rejects_small_workspace():

@@ -346,6 +346,56 @@ __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
 }  // namespace
 }  // namespace infv2
 
+namespace infv2 {
+namespace {
+
+// Stage 5 of the decode step: split-KV block-sparse attention of the query at
+// position pos[s] of each sequence; the last piece of a row writes pos + 1 to
+// pos_out[s] (the advanced length, or scratch when nothing may change).
+int launch_decode_attn(const infv2_params* p, const uint16_t* q, const uint16_t* kc,
+                       const uint16_t* vc, const int* pos, int* pos_out, int batch, int cap,
+                       const int* idx, uint8_t* ws, const DecodePlan& d, uint16_t* o, float* lse,
+                       cudaStream_t cs) {
+  CUtensorMap tm_k, tm_v;
+  const uint64_t rows = (uint64_t)batch * p->h_kv;
+  if (!make_tmap_3d(&tm_k, kc, 128, cap, rows, 256, (uint64_t)cap * 256, 64, 64, 1) ||
+      !make_tmap_3d(&tm_v, vc, 128, cap, rows, 256, (uint64_t)cap * 256, 64, 64, 1))
+    return INFV2_ERR_CUDA;
+  AttnArgs a{};
+  a.n_rows = batch;
+  a.h_q = p->h_q;
+  a.h_kv = p->h_kv;
+  a.k = p->k;
+  a.idx = idx;
+  a.idx_hstride = p->k;
+  a.idx_rstride = (long long)p->h_kv * p->k;
+  a.q = q;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.decode = 1;
+  a.seqlens = pos;
+  a.seqlens_out = pos_out;
+  a.cap = cap;
+  // as many pieces per row as keep the whole step in one wave of CTAs
+  int pieces = (2 * sm_count()) / (batch * p->h_kv);
+  if (pieces > kMaxPieces) pieces = kMaxPieces;
+  if (pieces > p->k) pieces = p->k;
+  if (pieces < 1) pieces = 1;
+  const int bps = (p->k + pieces - 1) / pieces;
+  a.n_split = (p->k + bps - 1) / bps;
+  a.blocks_per_split = bps;
+  a.split_out = 1;
+  a.part_o = reinterpret_cast<float*>(ws + d.off_po);
+  a.part_ml = reinterpret_cast<float*>(ws + d.off_pml);
+  a.counters = reinterpret_cast<int*>(ws + d.off_cnt);
+  a.o = o;
+  a.lse = lse;
+  a.wait = wait_ctx();
+  return launch_sparse_attn(tm_k, tm_v, a, cs);
+}
+
+}  // namespace
+}  // namespace infv2
+
 using namespace infv2;
 
 extern "C" int infv2_decode_workspace_size(const infv2_params* p, int batch, int cap,
@@ -429,42 +479,31 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     decode_select_kernel<<<dim3(kSelParts, batch * p->h_kv), 256, smem, cs>>>(a);
     if ((st = launch_status(cudaGetLastError())) != INFV2_OK) return st;
   }
-  {
-    CUtensorMap tm_k, tm_v;
-    const uint64_t rows = (uint64_t)batch * p->h_kv;
-    if (!make_tmap_3d(&tm_k, kc, 128, cap, rows, 256, (uint64_t)cap * 256, 64, 64, 1) ||
-        !make_tmap_3d(&tm_v, vc, 128, cap, rows, 256, (uint64_t)cap * 256, 64, 64, 1))
-      return INFV2_ERR_CUDA;
-    AttnArgs a{};
-    a.n_rows = batch;
-    a.h_q = p->h_q;
-    a.h_kv = p->h_kv;
-    a.k = p->k;
-    a.idx = idx;
-    a.idx_hstride = p->k;
-    a.idx_rstride = (long long)p->h_kv * p->k;
-    a.q = static_cast<const uint16_t*>(q);
-    a.scale_log2 = scale_log2;
-    a.decode = 1;
-    a.seqlens = seqlens;
-    a.seqlens_out = seqlens;
-    a.cap = cap;
-    // as many pieces per row as keep the whole step in one wave of CTAs
-    int pieces = (2 * sm_count()) / (batch * p->h_kv);
-    if (pieces > kMaxPieces) pieces = kMaxPieces;
-    if (pieces > p->k) pieces = p->k;
-    if (pieces < 1) pieces = 1;
-    const int bps = (p->k + pieces - 1) / pieces;
-    a.n_split = (p->k + bps - 1) / bps;
-    a.blocks_per_split = bps;
-    a.split_out = 1;
-    a.part_o = reinterpret_cast<float*>(ws + d.off_po);
-    a.part_ml = reinterpret_cast<float*>(ws + d.off_pml);
-    a.counters = counters;
-    a.o = static_cast<uint16_t*>(o);
-    a.lse = lse;
-    a.wait = wait_ctx();
-    if ((st = launch_sparse_attn(tm_k, tm_v, a, cs)) != INFV2_OK) return st;
-  }
-  return INFV2_OK;
+  return launch_decode_attn(p, static_cast<const uint16_t*>(q), kc, vc, seqlens, seqlens, batch,
+                            cap, idx, ws, d, static_cast<uint16_t*>(o), lse, cs);
+}
+
+extern "C" int infv2_decode_attn(const infv2_params* p, const void* q, const void* k_cache,
+                                 const void* v_cache, const int* pos, int batch, int cap,
+                                 const int* idx, void* workspace, size_t ws_bytes, void* o,
+                                 float* lse, infv2_stream_t stream) {
+  int st = infv2_check_params(p);
+  if (st != INFV2_OK) return st;
+  if (batch < 0 || cap <= 0) return INFV2_ERR_INVALID_ARG;
+  if (batch == 0) return INFV2_OK;
+  if (!q || !k_cache || !v_cache || !pos || !idx || !o) return INFV2_ERR_INVALID_ARG;
+  const DecodePlan d = plan_decode(p, batch, cap);
+  if (!workspace || ws_bytes < d.total) return INFV2_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return INFV2_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // the pieces' merge counters start at zero; the positions stay as given (the
+  // merge writes pos + 1 into the unused selection area of the workspace)
+  if (cudaMemsetAsync(ws + d.off_cnt, 0, (size_t)batch * (p->h_kv + 1) * 4, cs) != cudaSuccess)
+    return INFV2_ERR_CUDA;
+  return launch_decode_attn(p, static_cast<const uint16_t*>(q),
+                            static_cast<const uint16_t*>(k_cache),
+                            static_cast<const uint16_t*>(v_cache), pos,
+                            reinterpret_cast<int*>(ws + d.off_idx), batch, cap, idx, ws, d,
+                            static_cast<uint16_t*>(o), lse, cs);
 }

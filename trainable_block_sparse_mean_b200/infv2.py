@@ -26,7 +26,7 @@ SYMBOLS = [
     "infv2_compress_k2", "infv2_block_scores_approx", "infv2_sparse_attn_bwd_workspace_size",
     "infv2_sparse_attn_bwd", "infv2_pipeline_workspace_size", "infv2_pipeline_create",
     "infv2_pipeline_submit", "infv2_pipeline_wait", "infv2_pipeline_join", "infv2_pipeline_sync",
-    "infv2_pipeline_destroy", "infv2_sparse_attn_rows",
+    "infv2_pipeline_destroy", "infv2_sparse_attn_rows", "infv2_decode_attn",
 ]
 
 
@@ -79,6 +79,7 @@ def lib():
         L.infv2_prefill.argtypes = [P, vp, vp, vp, vp, i, vp, sz, vp, vp, vp, vp]
         L.infv2_decode_workspace_size.argtypes = [P, i, i, ctypes.POINTER(sz)]
         L.infv2_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i, i, vp, sz, vp, vp, vp, vp]
+        L.infv2_decode_attn.argtypes = [P, vp, vp, vp, vp, i, i, vp, vp, sz, vp, vp, vp]
         L.infv2_select_blocks_noalloc.argtypes = [P, vp, vp, i, i, i, vp, vp]
         L.infv2_selftest_timeout.argtypes = [i, vp]
         L.infv2_pipeline_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
@@ -415,6 +416,20 @@ def infv2_decode(p: Params, q, k_new, v_new, k_cache, v_cache, kc1_cache, seqlen
                               _ptr(v_cache), _ptr(kc1_cache), _ptr(seqlens), batch, cap,
                               _ptr(workspace), workspace.numel(), _ptr(idx_out), _ptr(o),
                               _ptr(lse), _stream(stream)), "infv2_decode")
+    return o
+
+
+def infv2_decode_attn(p: Params, q, k_cache, v_cache, pos, idx, workspace, o=None, lse=None,
+                      stream=None):
+    """Decode attention alone over given block lists idx [batch, h_kv, k] at
+    query positions pos (int32 [batch], device); caches and pos are not written."""
+    batch, cap = k_cache.shape[0], k_cache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().infv2_decode_attn(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(pos), batch, cap, _ptr(idx), _ptr(workspace),
+                                   workspace.numel(), _ptr(o), _ptr(lse), _stream(stream)),
+           "infv2_decode_attn")
     return o
 
 

@@ -155,10 +155,22 @@ def make_decode_sequence(shape: Shape, L: int, steps: int, seed: int, s: int) ->
     """History of sequence s (L cached tokens) plus `steps` new tokens.
 
     Returns k/v [L+steps, h_kv, d] (the first L rows are the cache, row L+t is
-    the token appended at decode step t) and q_new [steps, h_q, d].
+    the token appended at decode step t) and q_new [steps, h_q, d].  The same
+    value distributions as make_prefill (no needles), but only the queries of
+    the new tokens are drawn: a decode step never reads the history's queries.
+    Draw order: q_new, K noise, K block offsets, V, from seed [seed, 1000 + s].
     """
-    p = make_prefill(shape, seed=[seed, 1000 + s], n=L + steps, n_needles=0)
-    return dict(k=p["k"], v=p["v"], q_new=p["q"][L:L + steps], L=L)
+    rng = np.random.default_rng([seed, 1000 + s])
+    n = L + steps
+    h_kv, d, B = shape.h_kv, shape.d, shape.B
+    n_blk = (n + B - 1) // B
+    q_new = bf16_bits(_normal(rng, (steps, shape.h_q, d)))
+    kf = _normal(rng, (n, h_kv, d))
+    off = _normal(rng, (h_kv, max(n_blk, 1), d)) * np.float32(0.5)
+    for g in range(h_kv):
+        kf[:, g, :] += np.repeat(off[g], B, axis=0)[:n]
+    v = bf16_bits(_normal(rng, (n, h_kv, d)))
+    return dict(k=bf16_bits(kf), v=v, q_new=q_new, L=L)
 
 
 def make_decode(shape: Shape, batch: int, len_lo: int, len_hi: int, steps: int,
