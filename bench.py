@@ -323,6 +323,9 @@ def run_ours(args, rank, world, local_rank, dist):
     e2e = _end_to_end(args, infv2, torch, p, shape, data, cu, stream, dev, max_ranks)
     # ---- decode
     dec = _decode(args, infv2, torch, shape, rank, dev, stream, max_ranks, DecodeState)
+    # ---- the other configurations and dense attention (reported beside the headline)
+    cfgs = _other_configs(args, infv2, torch, dev, stream, rank)
+    dense = _dense_timing(args, infv2, torch, dev, stream)
     if infv2.infv2_device_status() != 0:
         raise RuntimeError("kernel error word set during the benchmark")
 
@@ -334,7 +337,7 @@ def run_ours(args, rank, world, local_rank, dist):
     # dominant kernel and its roofline
     dom = max(stage["per_kernel"], key=lambda kk: stage["per_kernel"][kk]["ms_per_step"])
     dk = stage["per_kernel"][dom]
-    unit_flops = {"score_kernel": work["score"], "sparse_attn_kernel": work["attn"],
+    unit_flops = {"score_kernel": work["score"], "attn_tc_kernel": work["attn"],
                   "select_kernel": None, "compress_k_kernel": None}[dom]
     if unit_flops is not None:
         per_launch = unit_flops / dk["launches_per_step"]
@@ -375,6 +378,8 @@ def run_ours(args, rank, world, local_rank, dist):
         "score_exp": _score_exp_of(n, p.h_q, stage, dev, clk),
         "e2e": e2e,
         "decode": dec,
+        "configs": cfgs,
+        "dense": dense,
         "gpu_launches": launches_per_step * args.steps,
         "peaks": peaks,
     }
@@ -401,7 +406,7 @@ def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, 
     off_sh = ((nc * p.h_kv * 256) + 255) // 256 * 256
     s_sh = ws[off_sh: off_sh + p.h_kv * chunk_rows * ld * 4].view(torch.float32).view(p.h_kv, chunk_rows, ld)
     idx = torch.empty((p.h_kv, n, p.k), dtype=torch.int32, device=q.device)
-    names = ["compress_k_kernel", "score_kernel", "select_kernel", "sparse_attn_kernel"]
+    names = ["compress_k_kernel", "score_kernel", "select_kernel", "attn_tc_kernel"]
 
     def one(record):
         evs = []
@@ -424,7 +429,7 @@ def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, 
             evs.append(("select_kernel", b, ev()))
         a = ev()
         infv2.infv2_sparse_attn(p, q, k, v, idx, o, lse)
-        evs.append(("sparse_attn_kernel", a, ev()))
+        evs.append(("attn_tc_kernel", a, ev()))
         return evs
 
     for _ in range(max(1, args.warmup)):
@@ -455,6 +460,103 @@ def _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream, 
     for nm in names:
         per[nm] = {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in per[nm].items()}
     return dict(per_kernel=per, ms_per_step=e0.elapsed_time(e1) / steps, idx=idx)
+
+
+def _timed(torch, stream, fn, warm, steps):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _prefill_figures(args, infv2, torch, dev, stream, shape, data, cu, flops, stages=True):
+    """Tokens/s and algorithmic TFLOP/s of infv2_prefill over one (varlen)
+    batch; with `stages`, the stage breakdown of a single sequence: selection
+    share and the attention kernel's TFLOP/s against the measured peak."""
+    from trainable_block_sparse_mean_b200.workloads import to_dev
+    p = infv2.params_of(shape)
+    q, k, v = to_dev(data["q"], dev), to_dev(data["k"], dev), to_dev(data["v"], dev)
+    ws = torch.empty(max(infv2.infv2_prefill_workspace_size(p, cu), 256), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.h_q, q.shape[0]), device=dev)
+    steps = max(3, min(args.steps, 10))
+    ms = _timed(torch, stream, lambda: infv2.infv2_prefill(p, q, k, v, cu, workspace=ws, o=o, lse=lse),
+                max(1, args.warmup), steps)
+    peaks = measured_peaks()
+    T = int(cu[-1])
+    out = {"tokens": T, "ms_per_step": round(ms, 4), "tokens_per_s": round(T / (ms / 1e3), 1),
+           "algorithmic_tflop": round(flops["total"] / 1e12, 4),
+           "tflops": round(flops["total"] / (ms / 1e3) / 1e12, 2),
+           "tflops_frac_of_peak": round(flops["total"] / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+    if stages:
+        st = _stage_breakdown(args, infv2, torch, p, shape, q, k, v, o, lse, ws, stream,
+                              _chunk_rows(p, shape.n))
+        per = st["per_kernel"]
+        sel = sum(per[x]["ms_per_step"] for x in ("compress_k_kernel", "score_kernel", "select_kernel"))
+        at = per["attn_tc_kernel"]["ms_per_step"]
+        out["selection_share"] = round(sel / st["ms_per_step"], 4)
+        out["stages_ms"] = {kk: per[kk]["ms_per_step"] for kk in per}
+        out["attention"] = {"kernel": "attn_tc_kernel", "ms": at,
+                            "tflops": round(flops["attn"] / (at / 1e3) / 1e12, 2),
+                            "frac": round(flops["attn"] / (at / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+    return out
+
+
+def _other_configs(args, infv2, torch, dev, stream, rank):
+    """The configurations besides the headline: the 2k and 32k single
+    sequences and the varlen dense/sparse switch sweep (its dense sequences,
+    n <= k*B, and its sparse ones timed apart as well as together)."""
+    out = {}
+    for name in ("prefill_2k", "prefill_32k"):
+        sh = synth.CONFIGS[name]["shape"]
+        data = synth.make_prefill(sh, seed=rank)
+        w = prefill_work(sh, sh.n)
+        out[name] = _prefill_figures(args, infv2, torch, dev, stream, sh, data, [0, sh.n],
+                                     dict(total=w["score"] + w["attn"], attn=w["attn"]))
+    cfg = synth.CONFIGS["varlen_sweep"]
+    sh = cfg["shape"]
+    lengths = list(cfg["lengths"])
+    sweep = {}
+    for part, lens in (("all", lengths), ("dense", [x for x in lengths if x <= sh.k * sh.B]),
+                       ("sparse", [x for x in lengths if x > sh.k * sh.B])):
+        data = synth.make_varlen(sh, lens, seed=rank)
+        tot = 0.0
+        for L in lens:
+            w = prefill_work(sh, L)
+            tot += w["score"] + w["attn"]
+        fig = _prefill_figures(args, infv2, torch, dev, stream, sh, data, list(data["cu_seqlens"]),
+                               dict(total=tot, attn=0.0), stages=False)
+        fig["lengths"] = lens
+        sweep[part] = fig
+    out["varlen_sweep"] = sweep
+    return out
+
+
+def _dense_timing(args, infv2, torch, dev, stream):
+    """Dense causal attention (infv2_dense_attn) over a 4096-token sequence at
+    h_q=32, h_kv=2: the kernel a sequence of at most k*B tokens takes."""
+    from trainable_block_sparse_mean_b200.workloads import to_dev
+    sh = synth.Shape(n=4096, h_q=32, h_kv=2, k=64)
+    data = synth.make_prefill(sh, seed=0)
+    p = infv2.params_of(sh)
+    q, k, v = to_dev(data["q"], dev), to_dev(data["k"], dev), to_dev(data["v"], dev)
+    o = torch.empty_like(q)
+    ms = _timed(torch, stream, lambda: infv2.infv2_dense_attn(p, q, k, v, o=o), max(3, args.warmup),
+                max(10, min(args.steps, 50)))
+    flops = prefill_work(sh, sh.n)["attn"]
+    peaks = measured_peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": "dense causal attention, n=4096, h_q=32, h_kv=2, d=128, bf16",
+            "kernel": "attn_tc_kernel", "us": round(ms * 1e3, 2),
+            "algorithmic_tflop": round(flops / 1e12, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4)}}
 
 
 def _fused_pool_timing(args, infv2, torch, p, shape, q, k, ws, stream, chunk_rows, stage):

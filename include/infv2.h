@@ -310,8 +310,8 @@ int infv2_pipeline_create(const infv2_params* p, const int* cu_seqlens_host, int
  * allocated and the inputs unchanged, and the outputs must not be read, until
  * infv2_pipeline_sync returns (or a stream given to infv2_pipeline_join has
  * passed that point).  Errors: INFV2_ERR_INVALID_ARG (NULL pointer),
- * INFV2_ERR_CUDA (a copy, event or launch failed; the pipeline should then
- * be destroyed). */
+ * INFV2_ERR_CUDA (a copy, event or launch failed part-way: the pipeline then
+ * refuses further submits with INFV2_ERR_CUDA and should be destroyed). */
 int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, const void* k_host,
                           const void* v_host, void* o_host, float* lse_host);
 
@@ -391,11 +391,23 @@ int infv2_decode_attn(const infv2_params* p, const void* q, const void* k_cache,
  * for one 128-token tile do not fit (h_kv * ld * 4 * 128 > 16 MiB, with
  * ld = max(num_kernels(n), 4*ceil(n/B)) rounded up to 32; e.g. n > 262144 at
  * h_kv = 2) return INFV2_ERR_UNSUPPORTED.  The first call on a device looks up
- * the array's device address (make it before any stream capture).  Every call
+ * the array's device address (make it before any stream capture), and so does
+ * the first call after the device's context changed (a device reset).  Every call
  * shares the array: calls that can overlap on the GPU race and must be
  * serialised by the caller. */
 int infv2_select_blocks_noalloc(const infv2_params* p, const void* q, const void* kc1, int n,
                                 int q_begin, int q_len, int* idx, infv2_stream_t stream);
+
+/* Self-test of the exponentials the kernels use: y[i] = 2^x[i] by
+ *   which = 0  the MUFU instruction (ex2.approx, flush to zero);
+ *   which = 1  the FMA-pipe polynomial of the score kernel (degree 5, relative
+ *              error below 2.3e-7; x below -127 gives 0);
+ *   which = 2  the FMA-pipe cubic of the attention's probabilities (relative
+ *              error below 1.1e-4 on [-126, 64]; x <= -127 gives exactly 0,
+ *              x above 64 gives 2^64).
+ * No counterpart in the paper: it lets a test hold each form to its bound.
+ * x, y: device fp32 [n].  INFV2_ERR_INVALID_ARG for another `which`. */
+int infv2_selftest_exp2(int which, const float* x, float* y, int n, infv2_stream_t stream);
 
 /* Self-test of the bounded-wait error path: launches one kernel that waits
  * on a barrier nobody arrives at, with the given limit in microseconds; the

@@ -117,6 +117,9 @@ def test_argument_errors_before_any_launch():
     assert L.infv2_decode(P, None, None, None, None, None, None, None, 0, 16, None, 0, None, None,
                           None, None) == infv2.OK
     assert L.infv2_selftest_timeout(0, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_selftest_exp2(3, None, None, 4, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_selftest_exp2(1, None, None, 0, None) == infv2.OK
+    assert L.infv2_selftest_exp2(1, None, None, 4, None) == infv2.ERR_INVALID_ARG
     # decode attention alone: an empty batch does nothing; bad shapes, missing
     # pointers and a small or misaligned workspace are refused before any launch
     assert L.infv2_decode_attn(P, None, None, None, None, 0, 16, None, None, 0, None, None, None) == infv2.OK

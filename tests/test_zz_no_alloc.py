@@ -73,6 +73,14 @@ def test_noalloc_row_range_and_limits():
     torch.cuda.synchronize()
     assert torch.equal(idx[:, 3000:8000], ref[:, 3000:8000])
     assert bool((idx[:, :3000] == -7).all()) and bool((idx[:, 8000:] == -7).all())
-    # beyond the fixed scratch (one 128-token tile of S^shared must fit in 16 MiB)
+    # beyond the fixed scratch (one 128-token tile of S^shared must fit in 16
+    # MiB): refused before any launch; the buffers have the sizes the call
+    # names, so even a launch could not read or write past them
     big = 300000
-    assert _noalloc(p, q, kc1, big, 0, 1, idx) == infv2.ERR_UNSUPPORTED
+    pb = infv2.params_of(synth.Shape(n=big, h_q=2, h_kv=2, k=16))
+    q_big = torch.zeros((big, 2, 128), dtype=torch.bfloat16, device="cuda")
+    kc1_big = torch.zeros((infv2.num_kernels(pb, big), 2, 128), dtype=torch.bfloat16, device="cuda")
+    idx_big = torch.full((2, big, 16), -7, dtype=torch.int32, device="cuda")
+    assert _noalloc(pb, q_big, kc1_big, big, 0, 1, idx_big) == infv2.ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert bool((idx_big == -7).all())

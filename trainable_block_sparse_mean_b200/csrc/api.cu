@@ -14,6 +14,7 @@ __device__ int g_error_word;  // first kernel failure on this device (0 = none)
 
 constexpr int kMaxDevices = 64;
 int* g_error_ptr[kMaxDevices];
+uintptr_t g_error_ctx[kMaxDevices];
 int g_sm_count[kMaxDevices];
 std::mutex g_mu;
 
@@ -24,14 +25,32 @@ int current_device() {
 }
 }  // namespace
 
+uintptr_t current_context() {
+  typedef CUresult (*GetCtxFn)(CUcontext*);
+  static GetCtxFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (GetCtxFn) nullptr;
+    return (GetCtxFn)p;
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return 0;
+  return reinterpret_cast<uintptr_t>(c);
+}
+
 int* error_word() {
   int dev = current_device();
   if (dev < 0) return nullptr;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_error_ptr[dev]) {
+  // a cached address belongs to the context that looked it up (a device reset
+  // makes a new one)
+  if (!g_error_ptr[dev] || g_error_ctx[dev] != current_context()) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
     g_error_ptr[dev] = static_cast<int*>(p);
+    g_error_ctx[dev] = current_context();
   }
   return g_error_ptr[dev];
 }
@@ -103,6 +122,22 @@ __global__ void timeout_selftest_kernel(WaitCtx w) {
   __syncthreads();
   if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0, w);  // nobody arrives
   __syncthreads();
+}
+// y[i] = 2^x[i] through one of the kernels' exponential forms (self-test).
+__global__ void exp2_selftest_kernel(int which, const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  float2 r;
+  if (which == 0) {
+    r = make_float2(fast_exp2(v.x), fast_exp2(v.y));
+  } else if (which == 1) {
+    r = exp2_fma2(v);
+  } else {
+    r = exp2_cubic2(v);
+  }
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
 }
 }  // namespace
 
@@ -176,6 +211,16 @@ int infv2_device_status(infv2_stream_t stream) {
   if (cudaMemsetAsync(w, 0, sizeof(int), s) != cudaSuccess) return INFV2_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return INFV2_ERR_CUDA;
   return host;
+}
+
+int infv2_selftest_exp2(int which, const float* x, float* y, int n, infv2_stream_t stream) {
+  if (which < 0 || which > 2 || n < 0) return INFV2_ERR_INVALID_ARG;
+  if (n == 0) return INFV2_OK;
+  if (!x || !y) return INFV2_ERR_INVALID_ARG;
+  const int threads = 256, pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                         reinterpret_cast<cudaStream_t>(stream)>>>(which, x, y, n);
+  return launch_status(cudaGetLastError());
 }
 
 int infv2_selftest_timeout(int limit_us, infv2_stream_t stream) {

@@ -5,20 +5,24 @@
 // returns O and the log-sum-exp.  MiniCPM4 blog (query/key granularity): the
 // query unit is one token, and the heads of a GQA group share its block set.
 //
-// B200 design.  A work item is one (kv head g, query token i): the G <= 16 query
-// heads of the group form a 16-row tile (the group is the only reuse a token's
-// private block set allows).  Each selected 64-token block of K and V (2 x 16
-// KB) is fetched by TMA into a 4-stage shared-memory ring by a producer warp;
-// four consumer warps each own 16 of the block's 64 keys and run
-// S = Q K^T and O += P V as m16n8k16 bf16 MMAs with fp32 accumulation and an
-// online softmax, then merge their partial (max, sum, O) through shared
-// memory.  The grid is persistent (one CTA per SM) and walks the items kv-head
-// by kv-head so that one head's K/V stays resident in L2.
+// Where it runs: the decode step (one query token per sequence), and prefill
+// with block lists at group sizes G <= 2 or with lists longer than the
+// tensor-core kernel stages ((128/G) * k > 2048 entries per tile); attn_tc.cu
+// takes every other prefill shape.  A work item is one (kv head g,
+// query token i): the G <= 16 query heads of the group form a 16-row tile (the
+// group is the only reuse a single token's block set allows).  Each selected
+// 64-token block of K and V (2 x 16 KB) is fetched by TMA into a 2-stage
+// shared-memory ring by a producer warp; four consumer warps each own 16 of the
+// block's 64 keys and run S = Q K^T and O += P V as m16n8k16 bf16 MMAs with
+// fp32 accumulation and an online softmax, then merge their partial (max, sum,
+// O) through shared memory.  Two CTAs share an SM (2 stages keep both in
+// shared memory); the grid is persistent (two CTAs per SM) and walks the items
+// kv head by kv head so that one head's K/V stays resident in L2.
 //
-// The same kernel serves the decode step: a row is then a sequence of a batch
-// (K/V in cache layout, query position from seqlens), and the block list can
-// be split so that several CTAs share one row; splits write unnormalised
-// partial outputs that a combine kernel merges.
+// In the decode step a row is a sequence of the batch (K/V in cache layout,
+// query position from seqlens), and the block list is cut so that several CTAs
+// share one row; the pieces write unnormalised partial outputs, and the last
+// piece of a row merges them and advances the row's length.
 #include "attn_sparse.cuh"
 #include "common.cuh"
 

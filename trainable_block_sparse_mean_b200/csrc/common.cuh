@@ -426,7 +426,11 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, 
 // Status of the last launch / runtime call as an infv2_status.
 int launch_status(cudaError_t e);
 
-// Device address of this device's kernel error word (set up once per device).
+// Identity of the calling thread's current CUDA context (0 if none or unknown).
+uintptr_t current_context();
+
+// Device address of this device's kernel error word (looked up once per device
+// and context).
 int* error_word();
 
 // Wall-time limit of every bounded wait inside a kernel (default 2 s).

@@ -95,6 +95,7 @@ struct infv2_pipeline {
   cudaEvent_t out_done[2] = {nullptr, nullptr};
   cudaEvent_t fence = nullptr;
   bool used[2] = {false, false};
+  bool failed = false;  // a submit failed part-way: its slot's queued work is unordered
   int next = 0;
   long long T = 0;
   int n_qparts = 0;
@@ -263,9 +264,10 @@ struct SubmitHooks final : PrefillHooks {
 
 }  // namespace
 
-extern "C" int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, const void* k_host,
-                                     const void* v_host, void* o_host, float* lse_host) {
-  if (!pl || !q_host || !k_host || !v_host || !o_host) return INFV2_ERR_INVALID_ARG;
+namespace {
+
+int submit_once(infv2_pipeline* pl, const void* q_host, const void* k_host, const void* v_host,
+                void* o_host, float* lse_host) {
   DeviceGuard guard(pl->device);
   if (!guard.ok) return INFV2_ERR_CUDA;
   const int b = pl->next;
@@ -300,6 +302,19 @@ extern "C" int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, con
   pl->used[b] = true;
   pl->next = b ^ 1;
   return INFV2_OK;
+}
+
+}  // namespace
+
+extern "C" int infv2_pipeline_submit(infv2_pipeline* pl, const void* q_host, const void* k_host,
+                                     const void* v_host, void* o_host, float* lse_host) {
+  if (!pl || !q_host || !k_host || !v_host || !o_host) return INFV2_ERR_INVALID_ARG;
+  // after a failed submit, the slot's events no longer order the copies and
+  // kernels already queued for it, so the pipeline takes no more work
+  if (pl->failed) return INFV2_ERR_CUDA;
+  const int st = submit_once(pl, q_host, k_host, v_host, o_host, lse_host);
+  if (st != INFV2_OK) pl->failed = true;
+  return st;
 }
 
 extern "C" int infv2_pipeline_wait(infv2_pipeline* pl, infv2_stream_t stream) {

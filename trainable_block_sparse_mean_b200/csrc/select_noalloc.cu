@@ -13,7 +13,8 @@
 // use the array's name as a device address; its address is looked up once per
 // device with cudaGetSymbolAddress (on the first call made on that device,
 // which therefore should come before any stream capture) and passed to the
-// kernels.  All calls share the array: calls that overlap on the GPU (other
+// kernels (again whenever the device's context has changed, e.g. after a
+// device reset).  All calls share the array: calls that overlap on the GPU (other
 // streams, other threads) race on it and must be serialised by the caller.
 // Nothing in it needs clearing: every element the selection reads is written
 // earlier in the same call.
@@ -31,9 +32,11 @@ static __device__ __align__(256) float g_noalloc_scratch[kScratchBytes / sizeof(
 
 constexpr int kMaxDevices = 64;
 float* g_scratch_addr[kMaxDevices];
+uintptr_t g_scratch_ctx[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of g_noalloc_scratch on the current device (looked up once).
+// Device address of g_noalloc_scratch on the current device (looked up once per
+// device and context: an address is only valid in the context it came from).
 float* scratch_address(int* status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -41,13 +44,14 @@ float* scratch_address(int* status) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != current_context()) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       *status = INFV2_ERR_CUDA;
       return nullptr;
     }
     g_scratch_addr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = current_context();
   }
   *status = INFV2_OK;
   return g_scratch_addr[dev];
@@ -73,7 +77,8 @@ extern "C" int infv2_select_blocks_noalloc(const infv2_params* p, const void* q,
   if (row_bytes * kMinRowsPerChunk > kScratchBytes) return INFV2_ERR_UNSUPPORTED;
   float* scratch = scratch_address(&st);
   if (!scratch) return st;
-  const int chunk = (int)(kScratchBytes / row_bytes);
+  // whole score tiles per chunk (128 rows): no chunk ends on a partial tile
+  const int chunk = (int)(kScratchBytes / row_bytes) / kMinRowsPerChunk * kMinRowsPerChunk;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const uint16_t* qb = static_cast<const uint16_t*>(q);
   const uint16_t* kb = static_cast<const uint16_t*>(kc1);

@@ -27,6 +27,7 @@ SYMBOLS = [
     "infv2_sparse_attn_bwd", "infv2_pipeline_workspace_size", "infv2_pipeline_create",
     "infv2_pipeline_submit", "infv2_pipeline_wait", "infv2_pipeline_join", "infv2_pipeline_sync",
     "infv2_pipeline_destroy", "infv2_sparse_attn_rows", "infv2_decode_attn",
+    "infv2_selftest_exp2",
 ]
 
 
@@ -82,6 +83,7 @@ def lib():
         L.infv2_decode_attn.argtypes = [P, vp, vp, vp, vp, i, i, vp, vp, sz, vp, vp, vp]
         L.infv2_select_blocks_noalloc.argtypes = [P, vp, vp, i, i, i, vp, vp]
         L.infv2_selftest_timeout.argtypes = [i, vp]
+        L.infv2_selftest_exp2.argtypes = [i, vp, vp, i, vp]
         L.infv2_pipeline_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
         L.infv2_pipeline_create.argtypes = [P, vp, i, vp, sz, vp, ctypes.POINTER(vp)]
         L.infv2_pipeline_submit.argtypes = [vp, vp, vp, vp, vp, vp]
@@ -441,6 +443,15 @@ def infv2_select_blocks_noalloc(p: Params, q, kc1, n: int, q_begin: int, q_len: 
                                              q_len, _ptr(idx), _stream(stream)),
            "infv2_select_blocks_noalloc")
     return idx
+
+
+def infv2_selftest_exp2(which: int, x, stream=None):
+    """2^x through one of the kernels' exponential forms (0: MUFU, 1: the
+    score kernel's degree-5 polynomial, 2: the attention's cubic)."""
+    y = torch.empty_like(x)
+    _check(lib().infv2_selftest_exp2(which, _ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "infv2_selftest_exp2")
+    return y
 
 
 def infv2_selftest_timeout(limit_us: int, stream=None):
