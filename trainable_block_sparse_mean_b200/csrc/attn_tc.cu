@@ -13,8 +13,9 @@
 // warp merges the lists and tags each union block with the mask of the tokens
 // that chose it.  Every union block's K and V (64 keys x 128 dims each) is
 // fetched once by TMA and serves all 128 rows:
-//   S  = Q K^T   tcgen05 M=128 N=64 K=128; A = Q in TMEM, B = K in shared memory
-//   softmax      one thread per row; rows whose token did not choose the block
+//   S  = Q K^T   tcgen05 M=128 N=64 per block, K=128; A = Q in TMEM, B = K in
+//                shared memory
+//   softmax      four threads per row; rows whose token did not choose the block
 //                get P = 0 (a warp with no such row only stores zeros)
 //   O += P V     tcgen05 M=128 N=128 K=64; A = P (bf16, written over S's
 //                columns) in TMEM, B = V in shared memory (MN-major)
@@ -31,24 +32,23 @@
 //    that each one's barrier waits overlap the other's issue;
 //  - S has two TMEM buffers of a pair each, so QK of the next pair runs while
 //    the softmax of this one does;
-//  - eight softmax warps, two per TMEM lane quarter, each take one block of a
-//    pair, so every SM sub-partition has a second warp to hide latency;
-//  - a row's reference max is set at its first chosen block and then kept; a
-//    pair takes the slow path (max of both blocks, O rescaled in TMEM) only when
-//    a block's probabilities sum past 2^16, so there is no per-block max; the
-//    two warps of a lane quarter agree on that through a bounded mbarrier
-//    exchange of one ballot per pair;
+//  - eight softmax warps, two per TMEM lane quarter, each own 16 rows (one
+//    token at G = 16) through the 16-lane TMEM load/store shapes, so a row's
+//    maximum and sum are reduced over four threads, and every SM sub-partition
+//    has a second warp to hide latency;
+//  - a row's reference max is raised only when a pair's max exceeds it by more
+//    than 8 (log2 units); O is then rescaled in TMEM, so most pairs skip it;
 //  - a quarter of the exponentials run on the FMA pipe (exp2_cubic2), and P is
 //    rounded to bf16 with integer adds and a byte permute.
-// Blocks a row did not choose add exact zeros, so a row's result does not
-// depend on the other tokens of its tile (a row-range launch gives the same
-// bits).  Q is double-buffered in TMEM: the next tile's QK products start
-// while this tile's O is read out.
+// Blocks a row did not choose add exact zeros.  The reference max of a row
+// depends on the pairs its tile walks, so a row's bits are the same in any
+// launch whose row range starts and ends on tile boundaries (multiples of
+// 128/G tokens); other cuts agree within rounding.  Q is double-buffered in
+// TMEM: the next tile's QK products start while this tile's O is read out.
 // Warp roles: warp 0 merges the lists, publishes the union pairs and loads Q
 // and K; warp 10 loads V; warp 1 issues the QK products and owns TMEM; warp 11
-// issues the PV products; warps 2-5 and 6-9 (first and second block of each
-// pair, one warp of each per TMEM lane quarter) copy Q into TMEM, run the
-// softmax and write O and the log-sum-exp.
+// issues the PV products; warps 2-9 copy Q into TMEM (2-5), run the softmax
+// and write O and the log-sum-exp.
 // Dense mode (no lists): a tile's union is every block up to its last token,
 // and causality alone masks.  The grid is persistent: CTA x takes tiles x,
 // x + gridDim.x, ..., ordered kv head by kv head (one head's K/V stays in L2)
