@@ -34,6 +34,12 @@
  *     stream) and return an infv2_status for argument / launch errors.  Errors
  *     detected inside a kernel (a bounded wait that timed out) are recorded in
  *     a per-device word read by infv2_device_status().
+ *   - Debug build: compiled with INFV2_CHECKS=1 (libinfv2_checks.so), the
+ *     kernels also check their data-dependent indices and invariants (block
+ *     lists ascending without repeats, each selected list's size, order and
+ *     forced blocks, finite attention results) and record INFV2_ERR_CHECK in
+ *     the same word on the first failure.  A check never traps and never
+ *     changes a result; the default build compiles them out.
  *   - No call retains a pointer after it returns, except a pipeline, which
  *     keeps its workspace and the host buffers of queued batches; calls that
  *     share output or workspace memory must be ordered on the caller's
@@ -57,7 +63,9 @@ enum infv2_status {
   INFV2_ERR_UNSUPPORTED = 2, /* valid for the method but not for this build's kernels */
   INFV2_ERR_WORKSPACE = 3,   /* workspace smaller than the *_workspace_size answer */
   INFV2_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
-  INFV2_ERR_TIMEOUT = 5      /* a kernel's bounded wait ran out (device word only) */
+  INFV2_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (device word only) */
+  INFV2_ERR_CHECK = 6        /* a device-side check of the INFV2_CHECKS build failed
+                                (device word only; never raised by the default build) */
 };
 
 /* Method parameters.
@@ -191,7 +199,11 @@ int infv2_select_topk_pooled(const infv2_params* p, const float* s_cmp, int ld_c
 
 /* Stage 5, block-sparse attention (arXiv summary, Appendix A): for every
  * query i and head h of group g, softmax attention over the tokens t <= i of
- * the blocks listed in idx[g, i, :] (entries < 0 ignored).
+ * the blocks listed in idx[g, i, :].  Entries < 0 and entries past the
+ * query's own block (i / 64) add nothing and are skipped; a row left with no
+ * block gets O = 0 and lse = -inf.  The lists are meant to be ascending
+ * without repeats, as infv2_select_topk writes them: a repeated block would
+ * count twice (the INFV2_CHECKS build reports that as INFV2_ERR_CHECK).
  *   q bf16 [n, h_q, d]; k, v bf16 [n, h_kv, d]; idx int32 [h_kv, n, k]
  *   o   bf16 [n, h_q, d] (output)
  *   lse fp32 [h_q, n] (output, nullable): natural log-sum-exp of the logits. */

@@ -35,6 +35,16 @@ def test_library_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_checks_build_exports_the_same_symbols():
+    # the INFV2_CHECKS debug variant is the same ABI with device-side checks
+    path = build_mod.build(checks=True)
+    lib = ctypes.CDLL(path)
+    missing = [s for s in declared_functions() if not hasattr(lib, s)]
+    assert not missing, missing
+    lib.infv2_status_string.restype = ctypes.c_char_p
+    assert b"INFV2_CHECKS" in lib.infv2_status_string(infv2.ERR_CHECK)
+
+
 def test_default_params_and_checks():
     p = infv2.params(32, 2)
     assert (p.B, p.l_c1, p.s_c1, p.pool_l, p.pool_s, p.d, p.k) == (64, 32, 16, 5, 4, 128, 64)

@@ -1,7 +1,10 @@
 """Build libinfv2.so in-tree: nvcc for sm_100a, one object per source in
 parallel, then a shared-library link with the static CUDA runtime.
 
-    python -m trainable_block_sparse_mean_b200.build [--force] [-j N]
+    python -m trainable_block_sparse_mean_b200.build [--force] [-j N] [--checks]
+
+--checks builds the debug variant libinfv2_checks.so (INFV2_CHECKS=1: device
+side index and invariant checks that record INFV2_ERR_CHECK, never trap).
 """
 from __future__ import annotations
 
@@ -17,6 +20,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libinfv2.so")
+BUILD_CHECKS = os.path.join(HERE, "_build_checks")
+LIB_CHECKS = os.path.join(HERE, "libinfv2_checks.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,11 +40,12 @@ def _deps():
     return max(os.path.getmtime(h) for h in hdrs)
 
 
-def _compile(src: str, force: bool, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, verbose: bool, checks: bool) -> str:
+    obj = os.path.join(BUILD_CHECKS if checks else BUILD, os.path.basename(src)[:-3] + ".o")
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), _deps()):
         return obj
-    cmd = [NVCC] + CFLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+    flags = CFLAGS + (["-DINFV2_CHECKS=1"] if checks else [])
+    cmd = [NVCC] + flags + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, r.stdout, r.stderr))
@@ -48,21 +54,25 @@ def _compile(src: str, force: bool, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
+          checks: bool = False) -> str:
+    """Build (if out of date) and return the path of the library: the default
+    build, or with checks=True the INFV2_CHECKS debug build."""
+    bdir, lib = (BUILD_CHECKS, LIB_CHECKS) if checks else (BUILD, LIB)
+    os.makedirs(bdir, exist_ok=True)
     srcs = sources()
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, verbose), srcs))
+        objs = list(ex.map(lambda s: _compile(s, force, verbose, checks), srcs))
     newest = max(os.path.getmtime(o) for o in objs)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        tmp = LIB + ".tmp%d" % os.getpid()
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < newest:
+        tmp = lib + ".tmp%d" % os.getpid()
         cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda"] * 0
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s\n%s" % (r.stdout, r.stderr))
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
@@ -70,5 +80,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-j", type=int, default=None)
     ap.add_argument("-v", action="store_true", help="print ptxas resource usage")
+    ap.add_argument("--checks", action="store_true", help="build the INFV2_CHECKS debug variant")
     a = ap.parse_args()
-    print(build(a.force, a.j, a.v))
+    print(build(a.force, a.j, a.v, a.checks))

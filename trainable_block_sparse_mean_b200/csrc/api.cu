@@ -192,6 +192,7 @@ const char* infv2_status_string(int status) {
     case INFV2_ERR_WORKSPACE: return "workspace too small";
     case INFV2_ERR_CUDA: return "CUDA error";
     case INFV2_ERR_TIMEOUT: return "kernel wait timed out";
+    case INFV2_ERR_CHECK: return "device-side check failed (INFV2_CHECKS build)";
     default: return "unknown status";
   }
 }

@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(160, 2)
         const int* row = a.idx ? a.idx + (size_t)g * a.idx_hstride + (size_t)i * a.k : nullptr;
         const int ne = row ? a.k : (i >> 6) + 1;
         for (int e = 0; e < ne; ++e) {
-          const int b = row ? __ldg(row + e) : e;
+          const int b = row ? list_block(row, e, i, a.wait.err) : e;
           if (b < 0) continue;
           const int s = (int)(pc % kDqStages);
           if (!mbar_wait(empty0 + 8 * s, (uint32_t)((pc / kDqStages) & 1) ^ 1u, a.wait)) {
@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(160, 2)
     bool ok = true;
     int chunk_b = 0;
     for (int e = 0; e < ne; ++e) {
-      if ((e & 31) == 0) chunk_b = e + lane < ne ? (row ? __ldg(row + e + lane) : e + lane) : -1;
+      if ((e & 31) == 0)
+        chunk_b = e + lane < ne ? (row ? list_block(row, e + lane, i, a.wait.err) : e + lane) : -1;
       const int b = __shfl_sync(0xFFFFFFFFu, chunk_b, e & 31);
       if (b < 0) continue;
       const int s = (int)(cc % kDqStages);

@@ -101,7 +101,9 @@ __device__ __forceinline__ void item_range(const AttnArgs& a, const Item& it, in
   }
 }
 
-__device__ __forceinline__ int block_at(const int* row, int e) { return row ? __ldg(row + e) : e; }
+__device__ __forceinline__ int block_at(const int* row, int e, int pos, int* err) {
+  return row ? list_block(row, e, pos, err) : e;
+}
 
 __global__ void __launch_bounds__(160, 2)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(160, 2)
         int e0, e1;
         item_range(a, it, pos, row, e0, e1);
         for (int e = e0; e < e1; ++e) {
-          const int b = block_at(row, e);
+          const int b = block_at(row, e, pos, a.wait.err);
           if (b < 0) continue;
           const int s = (int)(pc % kStages);
           if (!mbar_wait(empty0 + 8 * s, (uint32_t)((pc / kStages) & 1) ^ 1u, a.wait)) {
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(160, 2)
     int chunk_b = 0;
     for (int e = e0; e < e1; ++e) {
       if (((e - e0) & 31) == 0)  // next 32 entries of the list, one per lane
-        chunk_b = e + lane < e1 ? block_at(row, e + lane) : -1;
+        chunk_b = e + lane < e1 ? block_at(row, e + lane, pos, a.wait.err) : -1;
       const int b = __shfl_sync(0xFFFFFFFFu, chunk_b, (e - e0) & 31);
       if (b < 0) continue;
       const int s = (int)(cc % kStages);
@@ -420,6 +422,12 @@ __global__ void __launch_bounds__(160, 2)
           uint16_t* dst = a.o + ((size_t)it.r * a.h_q + h) * 128 + d0;
           reinterpret_cast<uint4*>(dst)[0] = w0;
           reinterpret_cast<uint4*>(dst)[1] = w1;
+          if (INFV2_CHECKS) {  // debug build: every output finite
+            bool fin = true;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) fin = fin && isfinite(acc[x] * inv);
+            check(fin, a.wait.err);
+          }
           if (a.lse && (t & 7) == 0)
             a.lse[(size_t)h * a.lse_ld + it.r] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         } else {
@@ -500,6 +508,12 @@ __global__ void __launch_bounds__(160, 2)
           uint16_t* dst = a.o + ((size_t)it.r * a.h_q + h) * 128 + d0;
           reinterpret_cast<uint4*>(dst)[0] = w0;
           reinterpret_cast<uint4*>(dst)[1] = w1;
+          if (INFV2_CHECKS) {  // debug build: every output finite
+            bool fin = true;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) fin = fin && isfinite(acc[x] * inv);
+            check(fin, a.wait.err);
+          }
           if (a.lse && (t & 7) == 0)
             a.lse[(size_t)it.r * a.h_q + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         }

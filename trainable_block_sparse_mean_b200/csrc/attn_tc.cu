@@ -271,14 +271,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; ok && b < b_hi; ++b) ok = entry(b, 0xFFFFFFFFu);
         if (ok) ok = close(b_hi, 0xFFFFFFFFu);
       } else {
-        // stage the tile's lists (tokens outside [lo, hi) get none)
+        // stage the tile's lists (tokens outside [lo, hi) get none; blocks past
+        // a token's own are dropped here, so no row takes a block it cannot see)
         const int L = TQ * a.k;
         for (int e = lane; e < L; e += 32) {
           const int tok = e / a.k;
           const int i = T.i0 + tok;
           S.list[e] = (i >= T.lo && i < T.hi)
-                          ? __ldg(a.idx + T.g * a.idx_hstride + (long long)i * a.idx_rstride +
-                                  (e - tok * a.k))
+                          ? list_block(a.idx + T.g * a.idx_hstride + (long long)i * a.idx_rstride,
+                                       e - tok * a.k, i, a.wait.err)
                           : -1;
         }
         __syncwarp();
@@ -640,6 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok_hi)
             *reinterpret_cast<uint32_t*>(d_hi + d) =
                 pack_bf16(ov[4 * j + 2] * inv_hi, ov[4 * j + 3] * inv_hi);
+          if (INFV2_CHECKS)  // debug build: every output finite
+            check((!ok_lo || (isfinite(ov[4 * j] * inv_lo) && isfinite(ov[4 * j + 1] * inv_lo))) &&
+                      (!ok_hi || (isfinite(ov[4 * j + 2] * inv_hi) && isfinite(ov[4 * j + 3] * inv_hi))),
+                  a.wait.err);
         }
       }
       if (tt == 0 && a.lse) {

@@ -19,6 +19,29 @@ __device__ __forceinline__ void report_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// The debug build (INFV2_CHECKS=1) adds device-side checks of data-dependent
+// indices and invariants.  A failed check records INFV2_ERR_CHECK and the
+// kernel carries on exactly as the default build would: a check never traps
+// and never changes a result.
+#ifndef INFV2_CHECKS
+#define INFV2_CHECKS 0
+#endif
+__device__ __forceinline__ void check(bool ok, int* err) {
+  if (INFV2_CHECKS && !ok) report_error(err, INFV2_ERR_CHECK);
+}
+
+// Entry e of a block list row as the attention kernels use it: entries < 0
+// and blocks past the query's own (no key t <= pos) are skipped (-1).  The
+// debug build checks that non-negative neighbours ascend (no repeats).
+__device__ __forceinline__ int list_block(const int* row, int e, int pos, int* err) {
+  const int x = __ldg(row + e);
+  if (INFV2_CHECKS && e > 0 && x >= 0) {
+    const int prev = __ldg(row + e - 1);
+    check(prev < x, err);
+  }
+  return x > (pos >> 6) ? -1 : x;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

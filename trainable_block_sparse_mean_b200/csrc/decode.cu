@@ -236,6 +236,7 @@ struct SelectDecArgs {
   int* part_cnt;     // [batch * h_kv]
   int* idx;          // [batch, h_kv, k]
   int n_keys;
+  int* err;          // device error word (debug-build checks)
 };
 
 // 2. selection for one (sequence, kv head), spread over kSelParts CTAs of 256
@@ -340,7 +341,7 @@ __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
   for (int b = t; b < n_cand; b += blockDim.x) keys[b] = __ldcg(kg + b);
   if (t == 0) a.part_cnt[sgi] = 0;
   __syncthreads();
-  select_topk_cta(keys, n_cand, a.k, hist, bcast, out);
+  select_topk_cta(keys, n_cand, a.k, hist, bcast, out, a.err);
 }
 
 }  // namespace
@@ -472,6 +473,7 @@ extern "C" int infv2_decode(const infv2_params* p, const void* q, const void* k_
     a.part_cnt = counters + (size_t)batch * (p->h_kv + 1);
     a.idx = idx;
     a.n_keys = d.n_keys;
+    a.err = error_word();
     const int part_kernels = 4 * ((d.n_keys + kSelParts - 1) / kSelParts) + 8;
     const int smem = (a.n_keys + 256 + 4 + 16 + part_kernels) * 4;
     if (smem > 200 * 1024) return INFV2_ERR_UNSUPPORTED;

@@ -13,6 +13,7 @@ struct SelectArgs {
   int* idx;               // idx[g * idx_hstride + i * k + :]
   long long idx_hstride;
   int keys_per_warp;      // shared words per warp for block keys
+  int* err;               // device error word (debug-build checks)
 };
 
 __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
@@ -27,7 +28,8 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   uint32_t* hist = keys + a.keys_per_warp;
   const float* row = a.s_shared + ((size_t)g * a.q_len + ii) * (size_t)a.ld;
   int* out = a.idx + (size_t)g * a.idx_hstride + (size_t)i * a.k;
-  select_row_warp(row, visible_kernels(i, 32, 16), i, a.n_init, a.n_local, a.k, keys, hist, out);
+  select_row_warp(row, visible_kernels(i, 32, 16), i, a.n_init, a.n_local, a.k, keys, hist, out,
+                  a.err);
 }
 
 // Top-k only, from S^cmp rows (max pooling already done by the score kernel).
@@ -43,7 +45,7 @@ __global__ void __launch_bounds__(256) select_pooled_kernel(SelectArgs a) {
   uint32_t* hist = keys + a.keys_per_warp;
   const float* row = a.s_shared + ((size_t)g * a.q_len + ii) * (size_t)a.ld;
   int* out = a.idx + (size_t)g * a.idx_hstride + (size_t)i * a.k;
-  select_row_warp_pooled(row, i, a.n_init, a.n_local, a.k, keys, hist, out);
+  select_row_warp_pooled(row, i, a.n_init, a.n_local, a.k, keys, hist, out, a.err);
 }
 
 template <typename Kernel>
@@ -59,7 +61,7 @@ int launch_select_rows(Kernel kernel, const infv2_params* p, const float* rows, 
   const int smem = warps * per_warp_bytes;
   if (!set_smem(kernel, smem)) return INFV2_ERR_CUDA;
   SelectArgs a{rows, ld, q_begin, q_len, p->h_kv, p->n_init, p->n_local, p->k,
-               idx, idx_hstride, keys_per_warp};
+               idx, idx_hstride, keys_per_warp, error_word()};
   const long long n_rows = (long long)p->h_kv * q_len;
   const long long blocks = (n_rows + warps - 1) / warps;
   kernel<<<(unsigned)blocks, warps * 32, smem, st>>>(a);

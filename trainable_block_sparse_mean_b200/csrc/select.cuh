@@ -27,8 +27,10 @@ constexpr uint32_t kForcedKey = 0xFFFFFFFFu;  // above every finite score and +i
 
 // Exact top-k of keys[0 .. n_cand) (per-warp shared memory) by one warp:
 // ascending block indices written to out[0..k), padded with -1.
+// The debug build (INFV2_CHECKS) checks that exactly k blocks come out (the
+// radix select's invariant) and writes none past k.
 __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int k, uint32_t* hist,
-                                          int* __restrict__ out) {
+                                          int* __restrict__ out, int* err) {
   const int lane = (int)lane_id();
   // ---- radix select of the k-th largest key
   uint32_t prefix = 0, pmask = 0;
@@ -92,9 +94,11 @@ __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int 
     const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
     eq_seen += __popc(eqb);
     const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
-    if (sel) out[written + __popc(selb & lt_mask)] = b;
+    const int at = written + __popc(selb & lt_mask);
+    if (sel && (!INFV2_CHECKS || at < k)) out[at] = b;
     written += __popc(selb);
   }
+  check(written == k, err);
   for (int x = written + lane; x < k; x += 32) out[x] = -1;
   __syncwarp();
 }
@@ -105,7 +109,7 @@ __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int 
 // Writes k indices (ascending, -1 padded) to `out`.
 __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, int nv, int i,
                                                 int n_init, int n_local, int k, uint32_t* keys,
-                                                uint32_t* hist, int* __restrict__ out) {
+                                                uint32_t* hist, int* __restrict__ out, int* err) {
   const int lane = (int)lane_id();
   const int bi = i >> 6;  // own block (B = 64)
   const int n_cand = bi + 1;
@@ -150,7 +154,7 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
     }
   }
   __syncwarp();
-  topk_warp(keys, n_cand, k, hist, out);
+  topk_warp(keys, n_cand, k, hist, out, err);
 }
 
 // Select for one row from precomputed block scores S^cmp[b] (b < i/B; the own
@@ -158,7 +162,7 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
 __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__ cmp, int i,
                                                        int n_init, int n_local, int k,
                                                        uint32_t* keys, uint32_t* hist,
-                                                       int* __restrict__ out) {
+                                                       int* __restrict__ out, int* err) {
   const int lane = (int)lane_id();
   const int bi = i >> 6;
   const int n_cand = bi + 1;
@@ -188,7 +192,7 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
     }
   }
   __syncwarp();
-  topk_warp(keys, n_cand, k, hist, out);
+  topk_warp(keys, n_cand, k, hist, out, err);
 }
 
 // Top-k over block keys already in shared memory (keys[0..bi], forced blocks
@@ -197,7 +201,7 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
 // Rows with at most k candidates are handled by the caller.
 __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand, int k,
                                                 uint32_t* hist, uint32_t* bcast,
-                                                int* __restrict__ out) {
+                                                int* __restrict__ out, int* err) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
   uint32_t prefix = 0, pmask = 0;
@@ -256,9 +260,11 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
       const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
       eq_seen += __popc(eqb);
       const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) out[written + __popc(selb & lt_mask)] = b;
+      const int at = written + __popc(selb & lt_mask);
+      if (sel && (!INFV2_CHECKS || at < k)) out[at] = b;
       written += __popc(selb);
     }
+    check(written == k, err);
     for (int x = written + lane; x < k; x += 32) out[x] = -1;
   }
 }

@@ -13,9 +13,12 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libinfv2.so")
+# INFV2_BUILD=checks loads the INFV2_CHECKS debug build (device-side index and
+# invariant checks) instead of the default one.
+LIB_PATH = os.path.join(_HERE, "libinfv2_checks.so" if os.environ.get("INFV2_BUILD") == "checks"
+                        else "libinfv2.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_CHECK = range(7)
 
 SYMBOLS = [
     "infv2_default_params", "infv2_check_params", "infv2_status_string", "infv2_num_kernels",
@@ -53,7 +56,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError("libinfv2.so not built: run python -m trainable_block_sparse_mean_b200.build")
+            raise ImportError("%s not built: run python -m trainable_block_sparse_mean_b200.build"
+                              % os.path.basename(LIB_PATH))
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.POINTER(Params)
         vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
