@@ -163,7 +163,8 @@ def test_pooled_block_scores_match_oracle(n, h_q, h_kv, q_begin, q_len):
             assert np.array_equal(got, pooled), (i, g)
 
 
-@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64)])
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64),
+                                         (3000, 4, 1, 3), (3000, 4, 1, 4)])
 def test_select_pooled_exact_on_oracle_scores(n, h_q, h_kv, k):
     """Top-k from S^cmp, decided on the same fp32 values as the oracle."""
     sh, d = _problem(n, h_q, h_kv, k=k, seed=4)
@@ -173,9 +174,10 @@ def test_select_pooled_exact_on_oracle_scores(n, h_q, h_kv, k):
     ref = oracle.prefill_rows(op, d["q"], d["k"], d["v"], rows, want_cmp=True)
     c32 = ref["cmp"].astype(np.float32)               # [rows, h_kv, n_blk]
     ties = np.round(c32 * 32) / 32
+    const = np.full_like(c32, 0.5)
     n_blk = c32.shape[2]
     ldc = infv2.cmp_ld(n)
-    for vals in (c32, ties):
+    for vals in (c32, ties, const):
         buf = np.full((h_kv, len(rows), ldc), np.nan, np.float32)
         for r, i in enumerate(rows):   # only b < i/B is defined; the rest stays NaN
             buf[:, r, :int(i) // 64] = vals[r, :, :int(i) // 64]
@@ -194,9 +196,12 @@ def test_select_pooled_exact_on_oracle_scores(n, h_q, h_kv, k):
 
 # ---------------------------------------------------------------- stages 3-4
 
-@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64)])
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(2048, 4, 1, 8), (5000, 32, 2, 16), (9000, 16, 2, 64),
+                                         (3000, 4, 1, 3), (3000, 4, 1, 4)])
 def test_select_exact_on_oracle_scores(n, h_q, h_kv, k):
-    """The selection decision is taken on the same fp32 values on both sides."""
+    """The selection decision is taken on the same fp32 values on both sides:
+    the scores as computed, a copy quantised to create many exact ties, and a
+    constant copy (every block tied); k = 3 leaves only the forced blocks."""
     sh, d = _problem(n, h_q, h_kv, k=k, seed=3)
     op = oracle.params(sh)
     p = infv2.params_of(sh)
@@ -206,7 +211,8 @@ def test_select_exact_on_oracle_scores(n, h_q, h_kv, k):
     nc = sh32.shape[2]
     # quantise a copy to create exact ties in the block scores
     ties = np.round(sh32 * 64) / 64
-    for vals in (sh32, ties):
+    const = np.full_like(sh32, 0.25)
+    for vals in (sh32, ties, const):
         ld = infv2.shared_ld(n)
         buf = np.zeros((h_kv, len(rows), ld), np.float32)
         buf[:, :, :nc] = vals.transpose(1, 0, 2)

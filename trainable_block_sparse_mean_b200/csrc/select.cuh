@@ -8,10 +8,13 @@
 //   I(i)     = every block 0..i/B when there are at most k of them; otherwise
 //              the init and local blocks (treated as +inf) plus the highest
 //              S^cmp blocks up to k in total, equal scores to the lower block.
-// The selection is an exact radix select on order-preserving 32-bit keys: four
-// 8-bit digit passes with a per-warp shared-memory histogram find the k-th
-// largest key T; blocks with key > T are taken, and the blocks with key == T
-// are taken in ascending block order until k are chosen.
+// The selection is an exact radix select on order-preserving 32-bit keys: up to
+// four 8-bit digit passes with a per-warp shared-memory histogram narrow down
+// the prefix T of the k-th largest key; blocks whose key prefix is above T are
+// taken, and the blocks with prefix T in ascending block order until k are
+// chosen.  The passes stop early once the bucket of the k-th key holds exactly
+// the number of blocks still needed (the whole bucket is then taken, which is
+// what the remaining passes would have found).
 #pragma once
 #include "common.cuh"
 
@@ -24,24 +27,42 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 }
 
 constexpr uint32_t kForcedKey = 0xFFFFFFFFu;  // above every finite score and +inf
+constexpr int kPoolLoads = 8;  // float4 loads in flight per lane while pooling a row
 
 // Exact top-k of keys[0 .. n_cand) (per-warp shared memory) by one warp:
-// ascending block indices written to out[0..k), padded with -1.
+// ascending block indices written to out[0..k), padded with -1.  The n_forced
+// keys equal to kForcedKey are always taken; the other keys lie in [kmin, kmax]
+// and compete for the remaining k - n_forced places.  They share every bit
+// above the highest bit in which kmin and kmax differ, so the digit passes
+// start there (on these scores the top byte is nearly constant, and a pass
+// over it would only pile every key into one bucket); each pass takes up to 8
+// bits.
 // The debug build (INFV2_CHECKS) checks that exactly k blocks come out (the
 // radix select's invariant) and writes none past k.
 __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int k, uint32_t* hist,
-                                          int* __restrict__ out, int* err) {
+                                          int* __restrict__ out, int* err, uint32_t kmin,
+                                          uint32_t kmax, int n_forced) {
   const int lane = (int)lane_id();
-  // ---- radix select of the k-th largest key
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = k;
+  // ---- radix select of the remaining-th largest non-forced key
+  int remaining = k - n_forced;
+  const uint32_t diff = kmin ^ kmax;
+  int top = diff ? 32 - __clz(diff) : 0;  // bits >= top are common to every competing key
+  uint32_t pmask = top >= 32 ? 0u : ~((1u << top) - 1u);
+  uint32_t prefix = kmin & pmask;
+  if (remaining <= 0) {  // only the forced blocks: no competing key can pass T
+    top = 0;
+    pmask = 0xFFFFFFFFu;
+    prefix = 0xFFFFFFFFu;
+  }
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (top > 0) {
+    const int shift = max(top - 8, 0);
+    const uint32_t dm = (1u << (top - shift)) - 1u;
     for (int x = lane; x < 256; x += 32) hist[x] = 0;
     __syncwarp();
     for (int b = lane; b < n_cand; b += 32) {
       const uint32_t key = keys[b];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if (key != kForcedKey && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dm], 1u);
     }
     __syncwarp();
     // lane L owns digits 255-8L .. 248-8L (lane 0 the largest)
@@ -60,7 +81,7 @@ __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int 
     }
     const uint32_t before = incl - local;
     const bool mine = before < (uint32_t)remaining && (uint32_t)remaining <= incl;
-    uint32_t digit = 0, above = 0;
+    uint32_t digit = 0, above = 0, dcnt = 0;
     if (mine) {
       uint32_t run = before;
 #pragma unroll
@@ -68,6 +89,7 @@ __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int 
         if (run + cnt[e] >= (uint32_t)remaining) {
           digit = 255u - 8u * lane - e;
           above = run;
+          dcnt = cnt[e];
           break;
         }
         run += cnt[e];
@@ -77,21 +99,28 @@ __device__ __forceinline__ void topk_warp(const uint32_t* keys, int n_cand, int 
     const int src = __ffs(who) - 1;
     digit = __shfl_sync(0xFFFFFFFFu, digit, src);
     above = __shfl_sync(0xFFFFFFFFu, above, src);
+    dcnt = __shfl_sync(0xFFFFFFFFu, dcnt, src);
     prefix |= digit << shift;
-    pmask |= 255u << shift;
+    pmask |= dm << shift;
     remaining -= (int)above;
+    top = shift;
     __syncwarp();
+    if (dcnt == (uint32_t)remaining) break;  // the whole bucket is taken
   }
-  // ---- emit ascending: key > T, then key == T in block order while needed
+  // ---- emit ascending: forced blocks and prefixes above T, then prefix T in
+  // block order while needed
   const uint32_t T = prefix;
   const uint32_t lt_mask = (1u << lane) - 1u;
   int eq_seen = 0, written = 0;
   for (int base = 0; base < n_cand; base += 32) {
     const int b = base + lane;
     const uint32_t key = b < n_cand ? keys[b] : 0u;
-    const bool eq = b < n_cand && key == T;
+    const bool forced = b < n_cand && key == kForcedKey;
+    const uint32_t m = key & pmask;
+    const bool eq = b < n_cand && !forced && m == T;
     const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
-    const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
+    const bool sel = forced || (b < n_cand && m > T) ||
+                     (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
     eq_seen += __popc(eqb);
     const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
     const int at = written + __popc(selb & lt_mask);
@@ -117,13 +146,14 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
     for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
     return;
   }
-  // ---- max pooling into order keys (forced blocks get the top key); four
-  // 512-byte row segments are loaded before any is used
+  // ---- max pooling into order keys (forced blocks get the top key);
+  // kPoolLoads 512-byte row segments are loaded before any is used
   float carry = -INFINITY;  // S^shared[4*base - 1] for the next chunk's lane 0
-  for (int base0 = 0; base0 < n_cand; base0 += 128) {
-    float4 vv[4];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // range of the non-forced keys
+  for (int base0 = 0; base0 < n_cand; base0 += 32 * kPoolLoads) {
+    float4 vv[kPoolLoads];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kPoolLoads; ++u) {
       const int b = base0 + 32 * u + lane;
       const int j0 = 4 * b;
       float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
@@ -139,7 +169,7 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
       vv[u] = v;
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kPoolLoads; ++u) {
       const int b = base0 + 32 * u + lane;
       const float4 v = vv[u];
       // kernel 4b-1 is the previous block's last kernel (lane-1's v.w)
@@ -149,12 +179,20 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
       if (b < n_cand) {
         const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
         const bool forced = b < n_init || b > bi - n_local;
-        keys[b] = forced ? kForcedKey : float_key(m);
+        const uint32_t key = float_key(m);
+        keys[b] = forced ? kForcedKey : key;
+        if (!forced) {
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
       }
     }
   }
+  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
   __syncwarp();
-  topk_warp(keys, n_cand, k, hist, out, err);
+  // n_cand > k >= n_init + n_local: the init and local sets are disjoint
+  topk_warp(keys, n_cand, k, hist, out, err, kmin, kmax, n_init + n_local);
 }
 
 // Select for one row from precomputed block scores S^cmp[b] (b < i/B; the own
@@ -170,6 +208,7 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
     for (int b = lane; b < k; b += 32) out[b] = b < n_cand ? b : -1;
     return;
   }
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // range of the non-forced keys
   for (int base = 0; base < n_cand; base += 128) {
     float4 vv;
     const int b0 = base + 4 * lane;
@@ -187,17 +226,24 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
       const int b = b0 + u;
       if (b < n_cand) {
         const bool forced = b < n_init || b > bi - n_local;
-        keys[b] = forced ? kForcedKey : float_key(v4[u]);
+        const uint32_t key = float_key(v4[u]);
+        keys[b] = forced ? kForcedKey : key;
+        if (!forced) {
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
       }
     }
   }
+  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
   __syncwarp();
-  topk_warp(keys, n_cand, k, hist, out, err);
+  topk_warp(keys, n_cand, k, hist, out, err, kmin, kmax, n_init + n_local);
 }
 
 // Top-k over block keys already in shared memory (keys[0..bi], forced blocks
-// holding kForcedKey), by a whole CTA: the same exact radix select as above
-// with a CTA-wide histogram.  `hist` 256 words, `bcast` 4 words (shared).
+// holding kForcedKey), by a whole CTA: an exact radix select from the top
+// byte, with the same early stop as above, on a CTA-wide histogram.  `hist` 256 words, `bcast` 4 words (shared).
 // Rows with at most k candidates are handled by the caller.
 __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand, int k,
                                                 uint32_t* hist, uint32_t* bcast,
@@ -236,6 +282,7 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
           if (run + cnt[e] >= (uint32_t)remaining) {
             bcast[0] = 255u - 8u * lane - e;
             bcast[1] = run;
+            bcast[2] = cnt[e];
             break;
           }
           run += cnt[e];
@@ -246,7 +293,9 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
     prefix |= bcast[0] << shift;
     pmask |= 255u << shift;
     remaining -= (int)bcast[1];
+    const bool done = bcast[2] == (uint32_t)remaining;  // the whole bucket is taken
     __syncthreads();
+    if (done) break;
   }
   if (warp == 0) {
     const uint32_t T = prefix;
@@ -254,7 +303,7 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
     int eq_seen = 0, written = 0;
     for (int base = 0; base < n_cand; base += 32) {
       const int b = base + lane;
-      const uint32_t key = b < n_cand ? keys[b] : 0u;
+      const uint32_t key = b < n_cand ? (keys[b] & pmask) : 0u;
       const bool eq = b < n_cand && key == T;
       const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
       const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
