@@ -241,11 +241,13 @@ def recorded_traffic(kernel: str):
         rec = json.load(f).get(kernel)
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
-        return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
-        return None
+    # one source file or a list of them (a kernel and the header that holds its body)
+    srcs = rec["source"] if isinstance(rec["source"], list) else [rec["source"]]
+    shas = rec["sha256"] if isinstance(rec["sha256"], list) else [rec["sha256"]]
+    for name, sha in zip(srcs, shas):
+        src = os.path.join(ROOT, name)
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != sha:
+            return None
     return rec
 
 

@@ -338,10 +338,32 @@ __global__ void __launch_bounds__(256) decode_select_kernel(SelectDecArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int b = t; b < n_cand; b += blockDim.x) keys[b] = __ldcg(kg + b);
+  if (t == 0) {
+    bcast[0] = 0xFFFFFFFFu;  // range of the competing (non-forced) keys
+    bcast[1] = 0u;
+  }
+  __syncthreads();
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int b = t; b < n_cand; b += blockDim.x) {
+    const uint32_t key = __ldcg(kg + b);
+    keys[b] = key;
+    if (key != kForcedKey) {
+      lo = min(lo, key);
+      hi = max(hi, key);
+    }
+  }
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  if ((t & 31) == 0) {
+    atomicMin(&bcast[0], lo);
+    atomicMax(&bcast[1], hi);
+  }
   if (t == 0) a.part_cnt[sgi] = 0;
   __syncthreads();
-  select_topk_cta(keys, n_cand, a.k, hist, bcast, out, a.err);
+  const uint32_t kmin = bcast[0], kmax = bcast[1];
+  __syncthreads();  // bcast is reused by the digit passes
+  // n_cand > k >= n_init + n_local: the init and local sets are disjoint
+  select_topk_cta(keys, n_cand, a.k, hist, bcast, out, a.err, kmin, kmax, a.n_init + a.n_local);
 }
 
 }  // namespace

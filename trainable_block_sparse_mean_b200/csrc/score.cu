@@ -23,8 +23,8 @@
 // columns (pass-1 row statistics are merged through shared memory).  A
 // quarter of the exponentials run on the FMA pipe (exp2_fma) so that the MUFU
 // unit is not the only pipe doing the softmax.
-// Accumulators are double-buffered in TMEM (2 x 128 columns) so the next
-// tile's MMA overlaps the current tile's epilogue.
+// Accumulators rotate through kAcc TMEM buffers of 128 columns so the next
+// tiles' MMAs overlap the current tile's epilogue.
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -32,6 +32,7 @@ namespace infv2 {
 namespace {
 
 constexpr int kStages = 4;
+constexpr int kAcc = 2;                    // TMEM accumulators of 128 columns
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kEpiWarps = 16;              // four epilogue warpgroups
 constexpr int kColGroups = kEpiWarps / 4;  // column groups of 128 / kColGroups columns
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_part = s_lse2 + 128;  // [column group][128 rows][max, sum]
   float* s_xch = s_part + kColGroups * 128 * 2;        // [3][kColGroups][4 quarters][TPG]
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_xch + 3 * kColGroups * 4 * TPG + 2);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 4 + kColGroups);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kStages + 2 * kAcc + kColGroups);
   ScoreSmem S;
   S.q = smem_u32(base);
   S.k = S.q + kTileBytes;
@@ -88,8 +89,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   S.kv_full = S.q_full + 8;
   S.kv_empty = S.kv_full + 8 * kStages;
   S.acc_full = S.kv_empty + 8 * kStages;
-  S.acc_empty = S.acc_full + 16;
-  S.lse_ready = S.acc_empty + 16;
+  S.acc_empty = S.acc_full + 8 * kAcc;
+  S.lse_ready = S.acc_empty + 8 * kAcc;
   const uint32_t cg_bar0 = S.lse_ready + 8;  // POOL: one barrier per column group
 
   const int warp = threadIdx.x >> 5;
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(S.kv_full + 8 * s, 1);
       mbar_init(S.kv_empty + 8 * s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kAcc; ++b) {
       mbar_init(S.acc_full + 8 * b, 1);
       mbar_init(S.acc_empty + 8 * b, kEpiWarps);
     }
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(s_tmem), 256);
+    tmem_alloc(smem_u32(s_tmem), 128 * kAcc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -172,9 +173,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int it = 0; ok && it < total_it; ++it) {
         const int s = it % kStages;
-        const int b = it & 1;
+        const int b = it % kAcc;
         if (!mbar_wait(S.kv_full + 8 * s, (it / kStages) & 1, a.wait)) break;
-        if (!mbar_wait(S.acc_empty + 8 * b, ((it >> 1) & 1) ^ 1, a.wait)) break;
+        if (!mbar_wait(S.acc_empty + 8 * b, ((it / kAcc) & 1) ^ 1, a.wait)) break;
         tc_fence_after();
         const uint32_t ks = S.k + s * kTileBytes;
         const uint32_t a_base = it < n_kt1 ? S.q : ks;  // pass 1: rows = Q; pass 2: rows = K^C1
@@ -190,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = it + 1;
       }
       // never free TMEM under a running MMA: wait (bounded) for the last commits
-      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
-        (void)mbar_wait(S.acc_full + 8 * (it & 1), (it >> 1) & 1, a.wait);
+      for (int it = issued > kAcc ? issued - kAcc : 0; it < issued; ++it)
+        (void)mbar_wait(S.acc_full + 8 * (it % kAcc), (it / kAcc) & 1, a.wait);
     }
   } else {
     // ---------------------------------------------------------- epilogue warps
@@ -222,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     for (int it = 0; it < total_it; ++it) {
-      const int b = it & 1;
-      if (!mbar_wait(S.acc_full + 8 * b, (it >> 1) & 1, a.wait)) break;
+      const int b = it % kAcc;
+      if (!mbar_wait(S.acc_full + 8 * b, (it / kAcc) & 1, a.wait)) break;
       tc_fence_after();
       float v[32];
       tmem_ld32(lane_base + b * 128, v);
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 128 * kAcc);
   }
 }
 
@@ -406,7 +407,7 @@ int launch_score_g(const ScoreLaunch& L, cudaStream_t st) {
   constexpr int TPG = kCols / G > 0 ? kCols / G : 1;
   const int smem = kTileBytes * (1 + kStages) + 128 * 4 + kColGroups * 128 * 2 * 4 +
                    (3 * kColGroups * 4 * TPG + 2) * 4 +
-                   8 * (2 + 2 * kStages + 4 + kColGroups) + 16 + 1024;
+                   8 * (2 + 2 * kStages + 2 * kAcc + kColGroups) + 16 + 1024;
   if (!set_smem(score_kernel<G, POOL>, smem)) return INFV2_ERR_CUDA;
   ScoreArgs a;
   a.q_begin = L.q_begin;

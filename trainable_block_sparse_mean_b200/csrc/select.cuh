@@ -242,23 +242,36 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
 }
 
 // Top-k over block keys already in shared memory (keys[0..bi], forced blocks
-// holding kForcedKey), by a whole CTA: an exact radix select from the top
-// byte, with the same early stop as above, on a CTA-wide histogram.  `hist` 256 words, `bcast` 4 words (shared).
-// Rows with at most k candidates are handled by the caller.
+// holding kForcedKey), by a whole CTA: the same exact radix select as
+// topk_warp (passes from the first bit in which the competing keys differ,
+// early stop) on a CTA-wide histogram.  kmin / kmax bound the n_forced-free
+// keys.  `hist` 256 words, `bcast` 4 words (shared).  Rows with at most k
+// candidates are handled by the caller.
 __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand, int k,
                                                 uint32_t* hist, uint32_t* bcast,
-                                                int* __restrict__ out, int* err) {
+                                                int* __restrict__ out, int* err, uint32_t kmin,
+                                                uint32_t kmax, int n_forced) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = k;
+  int remaining = k - n_forced;
+  const uint32_t diff = kmin ^ kmax;
+  int top = diff ? 32 - __clz(diff) : 0;
+  uint32_t pmask = top >= 32 ? 0u : ~((1u << top) - 1u);
+  uint32_t prefix = kmin & pmask;
+  if (remaining <= 0) {
+    top = 0;
+    pmask = 0xFFFFFFFFu;
+    prefix = 0xFFFFFFFFu;
+  }
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (top > 0) {
+    const int shift = max(top - 8, 0);
+    const uint32_t dm = (1u << (top - shift)) - 1u;
     for (int x = t; x < 256; x += blockDim.x) hist[x] = 0;
     __syncthreads();
     for (int b = t; b < n_cand; b += blockDim.x) {
       const uint32_t key = keys[b];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if (key != kForcedKey && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dm], 1u);
     }
     __syncthreads();
     if (warp == 0) {
@@ -291,9 +304,10 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
     }
     __syncthreads();
     prefix |= bcast[0] << shift;
-    pmask |= 255u << shift;
+    pmask |= dm << shift;
     remaining -= (int)bcast[1];
     const bool done = bcast[2] == (uint32_t)remaining;  // the whole bucket is taken
+    top = shift;
     __syncthreads();
     if (done) break;
   }
@@ -303,10 +317,13 @@ __device__ __forceinline__ void select_topk_cta(const uint32_t* keys, int n_cand
     int eq_seen = 0, written = 0;
     for (int base = 0; base < n_cand; base += 32) {
       const int b = base + lane;
-      const uint32_t key = b < n_cand ? (keys[b] & pmask) : 0u;
-      const bool eq = b < n_cand && key == T;
+      const uint32_t key = b < n_cand ? keys[b] : 0u;
+      const bool forced = b < n_cand && key == kForcedKey;
+      const uint32_t m = key & pmask;
+      const bool eq = b < n_cand && !forced && m == T;
       const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, eq);
-      const bool sel = (b < n_cand && key > T) || (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
+      const bool sel = forced || (b < n_cand && m > T) ||
+                       (eq && eq_seen + __popc(eqb & lt_mask) < remaining);
       eq_seen += __popc(eqb);
       const uint32_t selb = __ballot_sync(0xFFFFFFFFu, sel);
       const int at = written + __popc(selb & lt_mask);
