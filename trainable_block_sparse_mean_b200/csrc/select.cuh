@@ -209,28 +209,36 @@ __device__ __forceinline__ void select_row_warp_pooled(const float* __restrict__
     return;
   }
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // range of the non-forced keys
-  for (int base = 0; base < n_cand; base += 128) {
-    float4 vv;
-    const int b0 = base + 4 * lane;
-    if (b0 + 3 < bi) {
-      vv = __ldg(reinterpret_cast<const float4*>(cmp + b0));
-    } else {
-      vv.x = b0 + 0 < bi ? cmp[b0 + 0] : -INFINITY;
-      vv.y = b0 + 1 < bi ? cmp[b0 + 1] : -INFINITY;
-      vv.z = b0 + 2 < bi ? cmp[b0 + 2] : -INFINITY;
-      vv.w = b0 + 3 < bi ? cmp[b0 + 3] : -INFINITY;
-    }
-    const float v4[4] = {vv.x, vv.y, vv.z, vv.w};
+  // kPoolLoads float4 loads (4 blocks each) in flight per lane
+  for (int base = 0; base < n_cand; base += 128 * kPoolLoads) {
+    float4 vv[kPoolLoads];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = b0 + u;
-      if (b < n_cand) {
-        const bool forced = b < n_init || b > bi - n_local;
-        const uint32_t key = float_key(v4[u]);
-        keys[b] = forced ? kForcedKey : key;
-        if (!forced) {
-          kmin = min(kmin, key);
-          kmax = max(kmax, key);
+    for (int x = 0; x < kPoolLoads; ++x) {
+      const int b0 = base + 128 * x + 4 * lane;
+      if (b0 + 3 < bi) {
+        vv[x] = __ldg(reinterpret_cast<const float4*>(cmp + b0));
+      } else {
+        vv[x].x = b0 + 0 < bi ? cmp[b0 + 0] : -INFINITY;
+        vv[x].y = b0 + 1 < bi ? cmp[b0 + 1] : -INFINITY;
+        vv[x].z = b0 + 2 < bi ? cmp[b0 + 2] : -INFINITY;
+        vv[x].w = b0 + 3 < bi ? cmp[b0 + 3] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < kPoolLoads; ++x) {
+      const int b0 = base + 128 * x + 4 * lane;
+      const float v4[4] = {vv[x].x, vv[x].y, vv[x].z, vv[x].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int b = b0 + u;
+        if (b < n_cand) {
+          const bool forced = b < n_init || b > bi - n_local;
+          const uint32_t key = float_key(v4[u]);
+          keys[b] = forced ? kForcedKey : key;
+          if (!forced) {
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+          }
         }
       }
     }
