@@ -520,12 +520,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                   if (key > lim_hi) v[4 * j + 2 + e] = -INFINITY;
                 }
             }
-            float x_lo = -INFINITY, x_hi = -INFINITY;
+            // the 16 values of each row: eight three-operand maxima per row
+            float a_lo[4], a_hi[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              x_lo = fmaxf(x_lo, fmaxf(v[4 * j], v[4 * j + 1]));
-              x_hi = fmaxf(x_hi, fmaxf(v[4 * j + 2], v[4 * j + 3]));
+            for (int x = 0; x < 4; ++x) {
+              a_lo[x] = fmax3(v[8 * x], v[8 * x + 1], v[8 * x + 4]);
+              a_hi[x] = fmax3(v[8 * x + 2], v[8 * x + 3], v[8 * x + 6]);
             }
+            float x_lo = fmax3(fmax3(a_lo[0], a_lo[1], v[5]), fmax3(a_lo[2], a_lo[3], v[13]),
+                               fmax3(v[21], v[29], -INFINITY));
+            float x_hi = fmax3(fmax3(a_hi[0], a_hi[1], v[7]), fmax3(a_hi[2], a_hi[3], v[15]),
+                               fmax3(v[23], v[31], -INFINITY));
             if (t_lo) mx_lo = fmaxf(mx_lo, x_lo);
             if (t_hi) mx_hi = fmaxf(mx_hi, x_hi);
           };

@@ -240,12 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e)
             if (jb + e >= nv_r) v[e] = -INFINITY;
         }
-        float t4[4];
+        // the tile max of the row's 32 values: 16 three-operand maxima
+        float t3[11];
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-          t4[x] = fmaxf(fmaxf(fmaxf(v[x], v[x + 4]), fmaxf(v[x + 8], v[x + 12])),
-                        fmaxf(fmaxf(v[x + 16], v[x + 20]), fmaxf(v[x + 24], v[x + 28])));
-        const float cm = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
+        for (int x = 0; x < 10; ++x) t3[x] = fmax3(v[3 * x], v[3 * x + 1], v[3 * x + 2]);
+        t3[10] = fmaxf(v[30], v[31]);
+        const float u0 = fmax3(t3[0], t3[1], t3[2]), u1 = fmax3(t3[3], t3[4], t3[5]);
+        const float u2 = fmax3(t3[6], t3[7], t3[8]), u3 = fmaxf(t3[9], t3[10]);
+        const float cm = fmaxf(fmax3(u0, u1, u2), u3);
         if (cm > vmax) {
           l *= fast_exp2((vmax - cm) * c);
           vmax = cm;

@@ -177,7 +177,7 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ row, i
       if (lane == 0) prev = carry;
       carry = __shfl_sync(0xFFFFFFFFu, v.w, 31);
       if (b < n_cand) {
-        const float m = fmaxf(fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)), prev);
+        const float m = fmax3(fmax3(v.x, v.y, v.z), v.w, prev);
         const bool forced = b < n_init || b > bi - n_local;
         const uint32_t key = float_key(m);
         keys[b] = forced ? kForcedKey : key;
