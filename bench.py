@@ -264,6 +264,9 @@ def run_ours(args, rank, world, local_rank, dist):
         dec = _decode(args, infv2, torch, None, rank, dev, torch.cuda.current_stream(),
                       lambda x: x, DecodeState)
         return {"metric": METRIC, "decode": dec}
+    if args.only == "dense":    # profiling runs: the dense 4096-token attention only
+        return {"metric": METRIC, "dense": _dense_timing(args, infv2, torch, dev,
+                                                         torch.cuda.current_stream())}
     shape = synth.CONFIGS[args.workload]["shape"]
     n = shape.n
     p = infv2.params_of(shape)
@@ -845,8 +848,8 @@ def main():
                     help="prefill workload: prefill_128k (131072 tokens, the reported one) or prefill_32k (32768)")
     ap.add_argument("--decode-small", action="store_true",
                     help="with --only decode: 8 sequences of 16k-32k tokens (profiler runs)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
-                    help="prefill / decode / backward: time only that part (for profiler runs)")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward", "dense"], default="all",
+                    help="prefill / decode / backward / dense: time only that part (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
