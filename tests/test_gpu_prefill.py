@@ -82,7 +82,14 @@ def test_prefill_2k_every_row():
     assert st["equal"] + st["swapped"] == sh.n
 
 
-@pytest.mark.parametrize("n,h_q,h_kv,k", [(12345, 32, 2, 64), (5000, 16, 2, 16), (3000, 8, 1, 8)])
+@pytest.mark.parametrize("n,h_q,h_kv,k", [(12345, 32, 2, 64), (5000, 16, 2, 16), (3000, 8, 1, 8),
+                                         # k = 256, the largest supported: at G = 16 a tile's
+                                         # lists (8 tokens x 256) exactly fill the tensor-core
+                                         # kernel's staging buffer
+                                         (20000, 16, 1, 256),
+                                         # G = 4 with k = 128: 32 tokens x 128 entries overflow
+                                         # that buffer, so the per-token kernel runs instead
+                                         (10000, 4, 1, 128)])
 def test_medium_sizes(n, h_q, h_kv, k):
     sh = synth.Shape(n=n, h_q=h_q, h_kv=h_kv, k=k, n_needles=8)
     data = synth.make_prefill(sh, seed=7)
