@@ -394,9 +394,9 @@ def run_ours(args, rank, world, local_rank, dist):
 
 
 def _chunk_rows(p, n):
-    # mirrors the library's chunking of S^shared (256 MiB budget, multiples of 128 rows)
+    # mirrors the library's chunking of S^shared (1 GiB budget, multiples of 128 rows)
     ld = ((max((n - 32) // 16 + 1, 4 * ((n + 63) // 64)) + 31) // 32) * 32
-    rows = (256 << 20) // (p.h_kv * ld * 4)
+    rows = (1 << 30) // (p.h_kv * ld * 4)
     rows = max(128, (rows // 128) * 128)
     return min(rows, n)
 

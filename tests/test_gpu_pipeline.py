@@ -35,9 +35,9 @@ def _bits(t):
 @pytest.mark.parametrize("lengths,h_q,h_kv", [
     ([700, 300, 5000, 1300], 16, 2),
     ([2048], 16, 2),
-    # 20000 tokens at h_kv = 8: four score chunks, so the attention runs as four
+    # 40000 tokens at h_kv = 8: four score chunks, so the attention runs as four
     # row ranges between them (the single-launch device prefill is the reference)
-    ([20000, 300], 16, 8),
+    ([40000, 300], 16, 8),
 ])
 def test_pipeline_matches_device_prefill_and_oracle(lengths, h_q, h_kv):
     # k*B = 512: 300-token sequences are dense, the others sparse

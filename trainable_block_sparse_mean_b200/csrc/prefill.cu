@@ -11,7 +11,7 @@
 namespace infv2 {
 namespace {
 
-constexpr size_t kSharedChunkBytes = size_t(256) << 20;  // S^shared buffer budget
+constexpr size_t kSharedChunkBytes = size_t(1) << 30;  // S^shared buffer budget (1 GiB)
 
 struct PrefillPlan {
   int max_sparse_n = 0;
