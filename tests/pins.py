@@ -629,6 +629,24 @@ def pin_attend_empty_block_list():
     assert np.all(o == 0.0) and np.all(lse == -np.inf), (o, lse)
 
 
+def pin_attend_blocks_past_the_query_add_nothing():
+    """T(i) holds only tokens t <= i (arXiv summary, Appendix A; the causal
+    visible-token set): list entries past the query's own block, in range or
+    beyond the sequence, leave O and lse bit for bit as the list without them,
+    and a list of only such entries is the empty set (O = 0, lse = -inf)."""
+    sh, data = _small_problem(n=300, h_q=4, h_kv=2, d=16, seed=5, k=6)
+    p = oracle.params(sh)
+    i, g = 150, 0                    # own block 2; blocks 3, 4 are in range but later
+    base = [0, 1, 2, -1, -1, -1]
+    more = [0, 1, 2, 3, 4, 10 ** 6]
+    o0, l0 = oracle.attend_row(p, data["q"], data["k"], data["v"], i, g, base)
+    o1, l1 = oracle.attend_row(p, data["q"], data["k"], data["v"], i, g, more)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+    assert np.all(np.isfinite(l0))
+    o2, l2 = oracle.attend_row(p, data["q"], data["k"], data["v"], i, g, [3, 4, 10 ** 6, -1, -1, -1])
+    assert np.all(o2 == 0.0) and np.all(l2 == -np.inf), (o2, l2)
+
+
 def pin_maxpool_literal_window():
     """The literal reading of the max-pool window (kernels 4b .. 4b+4 of the
     visible ones; pool_rule = 1), by brute force, and that it differs from
