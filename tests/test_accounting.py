@@ -1,0 +1,48 @@
+"""The benchmark's accounting against brute force (CPU only).
+
+The roofline figures divide algorithmic work by measured time, so the work
+formulas in bench.py are pinned here against the method itself: the attention
+FLOPs against the visible keys of the oracle's own block lists, and the score
+chunking that bench.py mirrors against the library's workspace layout."""
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import oracle  # noqa: E402
+from trainable_block_sparse_mean_b200 import build as build_mod  # noqa: E402
+from trainable_block_sparse_mean_b200 import infv2, synth  # noqa: E402
+
+
+def test_attention_flops_match_the_oracle_lists():
+    # every row of a 3000-token sequence: 4*d FLOP per (head, selected visible key)
+    sh = synth.Shape(n=3000, h_q=4, h_kv=1, d=128, k=8)
+    data = synth.make_prefill(sh, seed=2)
+    rows = np.arange(sh.n, dtype=np.int32)
+    ref = oracle.prefill_rows(oracle.params(sh), data["q"], data["k"], data["v"], rows)
+    keys = 0
+    for r, i in enumerate(rows):
+        for b in (int(x) for x in ref["idx"][r, 0]):
+            if b >= 0:
+                keys += max(0, min(64 * b + 63, int(i)) - 64 * b + 1)
+    assert bench.prefill_work(sh, sh.n)["attn"] == 4 * sh.d * sh.h_q * keys
+
+
+def test_chunk_rows_mirror_the_library():
+    # the S^shared piece of the prefill workspace is one chunk of chunk_rows rows
+    build_mod.build()
+    for name in ("prefill_32k", "prefill_128k"):
+        sh = synth.CONFIGS[name]["shape"]
+        p = infv2.params_of(sh)
+        n = sh.n
+        ws = infv2.infv2_prefill_workspace_size(p, [0, n])
+        r256 = lambda x: (x + 255) // 256 * 256
+        nc = infv2.num_kernels(p, n)
+        rest = ws - r256(nc * p.h_kv * 256) - r256(p.h_kv * n * p.k * 4)
+        rows = bench._chunk_rows(p, n)
+        assert rest == r256(rows * p.h_kv * infv2.shared_ld(n) * 4), name
+        assert rows % 128 == 0 or rows == n
