@@ -46,3 +46,25 @@ def test_chunk_rows_mirror_the_library():
         rows = bench._chunk_rows(p, n)
         assert rest == r256(rows * p.h_kv * infv2.shared_ld(n) * 4), name
         assert rows % 128 == 0 or rows == n
+
+
+def test_decode_bytes_match_the_oracle_lists():
+    # one decode step at query position L per sequence: the visible K^C1 rows,
+    # the K and V rows of the selected visible keys, and q, o, the new K and V
+    sh = synth.Shape(n=0, h_q=4, h_kv=2, d=128, k=8)
+    p = oracle.params(sh)
+    lens = np.array([700, 1500, 3000], np.int32)
+    kc1_rows = keys = 0
+    for s, L in enumerate(int(x) for x in lens):
+        sq = synth.make_decode_sequence(sh, L, 1, 4, s)
+        q = np.zeros((L + 1, sh.h_q, sh.d), np.uint16)
+        q[L] = sq["q_new"][0]
+        ref = oracle.prefill_rows(p, q, sq["k"][:L + 1], sq["v"][:L + 1], np.array([L], np.int32))
+        kc1_rows += sh.h_kv * oracle.visible_kernels(p, L)
+        for g in range(sh.h_kv):
+            for b in (int(x) for x in ref["idx"][0, g]):
+                if b >= 0:
+                    keys += min(64 * b + 63, L) - 64 * b + 1
+    row = sh.d * 2
+    want = kc1_rows * row + keys * 2 * row + len(lens) * (2 * sh.h_q * row + 2 * 2 * sh.h_kv * row)
+    assert bench.decode_bytes(sh, lens) == want
