@@ -255,6 +255,42 @@ int infv2_sparse_attn_bwd(const infv2_params* p, const void* q, const void* k, c
 int infv2_dense_attn(const infv2_params* p, const void* q, const void* k, const void* v, int n,
                      void* o, float* lse, infv2_stream_t stream);
 
+/* ---- Varlen forms of the stage calls ----------------------------------------
+ * The stage calls above on a packed batch ("thd": q [T, h_q, d], k and v
+ * [T, h_kv, d], T = cu_seqlens_host[batch]); sequence s owns tokens
+ * cu_seqlens_host[s] .. cu_seqlens_host[s+1]-1.  cu_seqlens_host is a HOST
+ * int32 array [batch + 1], starting at 0 and non-decreasing (as for
+ * infv2_prefill: each sequence's length sets its grids).  Each call issues,
+ * per sequence, the launches of the single-sequence call, so a sequence's
+ * results equal that call's bit for bit.  Per-sequence tensors are packed:
+ *   K^C1      [sum_s nc_s, h_kv, d]: sequence s's kernels from row cu_kernels[s]
+ *             (infv2_varlen_kernel_offsets), nc_s = infv2_num_kernels(p, n_s)
+ *   S^shared  sequence s's [h_kv, n_s, ld] block at float offset
+ *             h_kv * ld * cu_seqlens_host[s]; ld >= the largest nc_s, multiple
+ *             of 4 (the whole buffer: h_kv * T * ld floats, 16-byte aligned)
+ *   idx       int32 [h_kv, T, k]; o bf16 [T, h_q, d]; lse fp32 [h_q, T] (nullable)
+ * Errors as for the single-sequence calls; a bad cu_seqlens_host is
+ * INFV2_ERR_INVALID_ARG before any launch. */
+
+/* cu_kernels_host[s] = sum over t < s of infv2_num_kernels(p, n_t), for
+ * s = 0 .. batch (HOST int32 [batch + 1], output).  Host only. */
+int infv2_varlen_kernel_offsets(const infv2_params* p, const int* cu_seqlens_host, int batch,
+                                int* cu_kernels_host);
+int infv2_compress_k_varlen(const infv2_params* p, const void* k, const int* cu_seqlens_host,
+                            int batch, void* kc1, infv2_stream_t stream);
+int infv2_block_scores_varlen(const infv2_params* p, const void* q, const void* kc1,
+                              const int* cu_seqlens_host, int batch, float* s_shared, int ld,
+                              infv2_stream_t stream);
+int infv2_select_topk_varlen(const infv2_params* p, const float* s_shared, int ld,
+                             const int* cu_seqlens_host, int batch, int* idx,
+                             infv2_stream_t stream);
+int infv2_sparse_attn_varlen(const infv2_params* p, const void* q, const void* k, const void* v,
+                             const int* idx, const int* cu_seqlens_host, int batch, void* o,
+                             float* lse, infv2_stream_t stream);
+int infv2_dense_attn_varlen(const infv2_params* p, const void* q, const void* k, const void* v,
+                            const int* cu_seqlens_host, int batch, void* o, float* lse,
+                            infv2_stream_t stream);
+
 /* Workspace bytes that infv2_prefill needs for this varlen batch.
  *   cu_seqlens_host  HOST int32 [batch + 1], cu_seqlens_host[0] = 0. */
 int infv2_prefill_workspace_size(const infv2_params* p, const int* cu_seqlens_host, int batch,

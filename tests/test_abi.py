@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from trainable_block_sparse_mean_b200 import build as build_mod
@@ -213,3 +214,34 @@ def test_binding_refuses_host_tensors():
     kv = torch.zeros((64, 1, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         infv2.infv2_dense_attn(p, q, kv, kv, o=q)
+
+
+def test_varlen_kernel_offsets_and_argument_errors():
+    p = infv2.params(16, 2, k=8)
+    cu = [0, 10, 100, 100, 5000]
+    ck = infv2.infv2_varlen_kernel_offsets(p, cu)
+    nc = [infv2.num_kernels(p, b - a) for a, b in zip(cu[:-1], cu[1:])]
+    assert ck == [0] + list(np.cumsum(nc))
+    assert nc[0] == 0 and nc[2] == 0
+    L = infv2.lib()
+    pp = ctypes.byref(p)
+    arr = lambda xs: (ctypes.c_int * len(xs))(*xs)
+    bad = [arr([5, 10]), arr([0, 10, 4])]          # must start at 0; must not decrease
+    for c in bad:
+        assert L.infv2_varlen_kernel_offsets(pp, c, 2 if len(c) == 3 else 1, arr([0, 0, 0])) == infv2.ERR_INVALID_ARG
+        nb = len(c) - 1
+        assert L.infv2_compress_k_varlen(pp, None, c, nb, None, None) == infv2.ERR_INVALID_ARG
+        assert L.infv2_block_scores_varlen(pp, None, None, c, nb, None, 32, None) == infv2.ERR_INVALID_ARG
+        assert L.infv2_select_topk_varlen(pp, None, 32, c, nb, None, None) == infv2.ERR_INVALID_ARG
+        assert L.infv2_sparse_attn_varlen(pp, None, None, None, None, c, nb, None, None, None) == infv2.ERR_INVALID_ARG
+        assert L.infv2_dense_attn_varlen(pp, None, None, None, c, nb, None, None, None) == infv2.ERR_INVALID_ARG
+    good = arr([0, 100, 3000])
+    # missing tensors, and an S^shared pitch below the longest sequence's kernel count
+    assert L.infv2_compress_k_varlen(pp, None, good, 2, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_block_scores_varlen(pp, None, None, good, 2, None, 64, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_select_topk_varlen(pp, None, 32, good, 2, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_sparse_attn_varlen(pp, None, None, None, None, good, 2, None, None, None) == infv2.ERR_INVALID_ARG
+    assert L.infv2_dense_attn_varlen(pp, None, None, None, good, 2, None, None, None) == infv2.ERR_INVALID_ARG
+    # an empty batch (or only empty sequences) does nothing and succeeds
+    assert L.infv2_sparse_attn_varlen(pp, None, None, None, None, arr([0, 0]), 1, None, None, None) == infv2.OK
+    assert L.infv2_compress_k_varlen(pp, None, arr([0]), 0, None, None) == infv2.OK

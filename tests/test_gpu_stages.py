@@ -354,3 +354,50 @@ def test_timeout_path_reports_and_recovers():
     assert infv2.infv2_device_status() == 0     # cleared
     x = torch.ones(4, device="cuda") * 2        # the context is still usable
     assert float(x.sum()) == 8.0
+
+
+# ---------------------------------------------------------------- varlen stage forms
+
+def test_varlen_stage_calls_equal_the_single_sequence_calls():
+    """Each varlen stage call issues, per sequence, the single-sequence call's
+    launches on the packed tensors: a sequence's K^C1, S^shared block, block
+    lists, O and lse equal the single-sequence results bit for bit (an empty
+    sequence, one without a complete kernel, a dense-sized and two sparse
+    ones; two kv heads, so the packed head strides differ from the
+    per-sequence ones)."""
+    sh = synth.Shape(n=0, h_q=16, h_kv=2, k=8)
+    lengths = [300, 2000, 0, 5000, 31]
+    d = synth.make_varlen(sh, lengths, seed=9)
+    p = infv2.params_of(sh)
+    q, k, v = to_dev(d["q"]), to_dev(d["k"]), to_dev(d["v"])
+    cu = [int(x) for x in synth.cu_seqlens_of(lengths)]
+    T = cu[-1]
+    ck = infv2.infv2_varlen_kernel_offsets(p, cu)
+    kc1 = infv2.infv2_compress_k_varlen(p, k, cu)
+    s_sh, ld = infv2.infv2_block_scores_varlen(p, q, kc1, cu)
+    idx = infv2.infv2_select_topk_varlen(p, s_sh, ld, cu)
+    lse = torch.full((sh.h_q, T), 7.0, device="cuda")
+    o = infv2.infv2_sparse_attn_varlen(p, q, k, v, idx, cu, lse=lse)
+    lse_d = torch.full((sh.h_q, T), 7.0, device="cuda")
+    od = infv2.infv2_dense_attn_varlen(p, q, k, v, cu, lse=lse_d)
+    torch.cuda.synchronize()
+    assert infv2.infv2_device_status() == 0
+    for s, n in enumerate(lengths):
+        if n == 0:
+            continue
+        a, b = cu[s], cu[s + 1]
+        qs, ks, vs = q[a:b].contiguous(), k[a:b].contiguous(), v[a:b].contiguous()
+        kc1_s = infv2.infv2_compress_k(p, ks)
+        assert ck[s + 1] - ck[s] == kc1_s.shape[0]
+        assert torch.equal(kc1[ck[s]:ck[s + 1]], kc1_s), s
+        s_s = infv2.infv2_block_scores(p, qs, kc1_s, n, 0, n, ld=ld)
+        blk = s_sh[sh.h_kv * ld * a: sh.h_kv * ld * b].view(sh.h_kv, n, ld)
+        assert torch.equal(blk, s_s), s
+        idx_s = infv2.infv2_select_topk(p, s_s, ld, n, 0, n)
+        assert torch.equal(idx[:, a:b], idx_s), s
+        lse_s = torch.empty((sh.h_q, n), device="cuda")
+        o_s = infv2.infv2_sparse_attn(p, qs, ks, vs, idx_s, lse=lse_s)
+        assert torch.equal(o[a:b], o_s) and torch.equal(lse[:, a:b], lse_s), s
+        lse_ds = torch.empty((sh.h_q, n), device="cuda")
+        od_s = infv2.infv2_dense_attn(p, qs, ks, vs, lse=lse_ds)
+        assert torch.equal(od[a:b], od_s) and torch.equal(lse_d[:, a:b], lse_ds), s

@@ -30,7 +30,9 @@ SYMBOLS = [
     "infv2_sparse_attn_bwd", "infv2_pipeline_workspace_size", "infv2_pipeline_create",
     "infv2_pipeline_submit", "infv2_pipeline_wait", "infv2_pipeline_join", "infv2_pipeline_sync",
     "infv2_pipeline_destroy", "infv2_sparse_attn_rows", "infv2_decode_attn",
-    "infv2_selftest_exp2",
+    "infv2_selftest_exp2", "infv2_varlen_kernel_offsets", "infv2_compress_k_varlen",
+    "infv2_block_scores_varlen", "infv2_select_topk_varlen", "infv2_sparse_attn_varlen",
+    "infv2_dense_attn_varlen",
 ]
 
 
@@ -88,6 +90,12 @@ def lib():
         L.infv2_select_blocks_noalloc.argtypes = [P, vp, vp, i, i, i, vp, vp]
         L.infv2_selftest_timeout.argtypes = [i, vp]
         L.infv2_selftest_exp2.argtypes = [i, vp, vp, i, vp]
+        L.infv2_varlen_kernel_offsets.argtypes = [P, vp, i, vp]
+        L.infv2_compress_k_varlen.argtypes = [P, vp, vp, i, vp, vp]
+        L.infv2_block_scores_varlen.argtypes = [P, vp, vp, vp, i, vp, i, vp]
+        L.infv2_select_topk_varlen.argtypes = [P, vp, i, vp, i, vp, vp]
+        L.infv2_sparse_attn_varlen.argtypes = [P, vp, vp, vp, vp, vp, i, vp, vp, vp]
+        L.infv2_dense_attn_varlen.argtypes = [P, vp, vp, vp, vp, i, vp, vp, vp]
         L.infv2_pipeline_workspace_size.argtypes = [P, vp, i, ctypes.POINTER(sz)]
         L.infv2_pipeline_create.argtypes = [P, vp, i, vp, sz, vp, ctypes.POINTER(vp)]
         L.infv2_pipeline_submit.argtypes = [vp, vp, vp, vp, vp, vp]
@@ -460,3 +468,77 @@ def infv2_selftest_exp2(which: int, x, stream=None):
 
 def infv2_selftest_timeout(limit_us: int, stream=None):
     _check(lib().infv2_selftest_timeout(limit_us, _stream(stream)), "infv2_selftest_timeout")
+
+
+# ------------------------------------------------------------ varlen stage forms
+# cu_seqlens: a host sequence of batch + 1 offsets (packed "thd" tensors).
+
+def infv2_varlen_kernel_offsets(p: Params, cu_seqlens):
+    cu = _cu_array(cu_seqlens)
+    out = (ctypes.c_int * len(cu_seqlens))()
+    _check(lib().infv2_varlen_kernel_offsets(ctypes.byref(p), ctypes.cast(cu, ctypes.c_void_p),
+                                             len(cu_seqlens) - 1, ctypes.cast(out, ctypes.c_void_p)),
+           "infv2_varlen_kernel_offsets")
+    return list(out)
+
+
+def infv2_compress_k_varlen(p: Params, k, cu_seqlens, kc1=None, stream=None):
+    """K^C1 of every sequence, packed: sequence s's kernels from row cu_kernels[s]."""
+    ck = infv2_varlen_kernel_offsets(p, cu_seqlens)
+    if kc1 is None:
+        kc1 = torch.empty((max(ck[-1], 1), p.h_kv, 128), dtype=torch.bfloat16, device=k.device)
+    cu = _cu_array(cu_seqlens)
+    _check(lib().infv2_compress_k_varlen(ctypes.byref(p), _ptr(k), ctypes.cast(cu, ctypes.c_void_p),
+                                         len(cu_seqlens) - 1, _ptr(kc1), _stream(stream)),
+           "infv2_compress_k_varlen")
+    return kc1
+
+
+def infv2_block_scores_varlen(p: Params, q, kc1, cu_seqlens, s_shared=None, ld=None, stream=None):
+    """S^shared of every row; sequence s's [h_kv, n_s, ld] block at float
+    offset h_kv*ld*cu_seqlens[s] of a flat buffer.  Returns (s_shared, ld)."""
+    n_max = max((b - a for a, b in zip(cu_seqlens[:-1], cu_seqlens[1:])), default=0)
+    if ld is None:
+        ld = shared_ld(n_max)
+    T = int(cu_seqlens[-1])
+    if s_shared is None:
+        s_shared = torch.zeros(max(p.h_kv * T * ld, 4), dtype=torch.float32, device=q.device)
+    cu = _cu_array(cu_seqlens)
+    _check(lib().infv2_block_scores_varlen(ctypes.byref(p), _ptr(q), _ptr(kc1),
+                                           ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1,
+                                           _ptr(s_shared), ld, _stream(stream)),
+           "infv2_block_scores_varlen")
+    return s_shared, ld
+
+
+def infv2_select_topk_varlen(p: Params, s_shared, ld: int, cu_seqlens, idx=None, stream=None):
+    T = int(cu_seqlens[-1])
+    if idx is None:
+        idx = torch.empty((p.h_kv, T, p.k), dtype=torch.int32, device=s_shared.device)
+    cu = _cu_array(cu_seqlens)
+    _check(lib().infv2_select_topk_varlen(ctypes.byref(p), _ptr(s_shared), ld,
+                                          ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1,
+                                          _ptr(idx), _stream(stream)), "infv2_select_topk_varlen")
+    return idx
+
+
+def infv2_sparse_attn_varlen(p: Params, q, k, v, idx, cu_seqlens, o=None, lse=None, stream=None):
+    if o is None:
+        o = torch.empty_like(q)
+    cu = _cu_array(cu_seqlens)
+    _check(lib().infv2_sparse_attn_varlen(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                          ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1,
+                                          _ptr(o), _ptr(lse), _stream(stream)),
+           "infv2_sparse_attn_varlen")
+    return o
+
+
+def infv2_dense_attn_varlen(p: Params, q, k, v, cu_seqlens, o=None, lse=None, stream=None):
+    if o is None:
+        o = torch.empty_like(q)
+    cu = _cu_array(cu_seqlens)
+    _check(lib().infv2_dense_attn_varlen(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                         ctypes.cast(cu, ctypes.c_void_p), len(cu_seqlens) - 1,
+                                         _ptr(o), _ptr(lse), _stream(stream)),
+           "infv2_dense_attn_varlen")
+    return o
