@@ -121,8 +121,12 @@ const char* infv2_status_string(int status);
 int infv2_num_kernels(const infv2_params* p, int n);
 
 /* Read and clear this device's kernel error word (waits for `stream`).
- * Returns INFV2_OK, INFV2_ERR_TIMEOUT, or INFV2_ERR_CUDA if the read fails. */
+ * Returns INFV2_OK, INFV2_ERR_TIMEOUT, INFV2_ERR_CHECK (debug build only), or
+ * INFV2_ERR_CUDA if the read fails. */
 int infv2_device_status(infv2_stream_t stream);
+
+/* The same call under a second name, infv2_get_device_status. */
+int infv2_get_device_status(infv2_stream_t stream);
 
 /* Stage 1 (paper notes, key design 3): K^C1[j, g, :] = bf16 round-to-nearest-
  * even of the exact mean of K[t, g, :] over t = j*s_c1 .. j*s_c1 + l_c1 - 1.

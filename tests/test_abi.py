@@ -245,3 +245,10 @@ def test_varlen_kernel_offsets_and_argument_errors():
     # an empty batch (or only empty sequences) does nothing and succeeds
     assert L.infv2_sparse_attn_varlen(pp, None, None, None, None, arr([0, 0]), 1, None, None, None) == infv2.OK
     assert L.infv2_compress_k_varlen(pp, None, arr([0]), 0, None, None) == infv2.OK
+
+
+def test_device_status_second_name():
+    # both names are the same call (no GPU here: both report the failed read)
+    L = infv2.lib()
+    a, b = L.infv2_device_status(None), L.infv2_get_device_status(None)
+    assert a == b

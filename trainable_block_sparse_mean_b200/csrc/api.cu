@@ -214,6 +214,8 @@ int infv2_device_status(infv2_stream_t stream) {
   return host;
 }
 
+int infv2_get_device_status(infv2_stream_t stream) { return infv2_device_status(stream); }
+
 int infv2_selftest_exp2(int which, const float* x, float* y, int n, infv2_stream_t stream) {
   if (which < 0 || which > 2 || n < 0) return INFV2_ERR_INVALID_ARG;
   if (n == 0) return INFV2_OK;

@@ -32,7 +32,7 @@ SYMBOLS = [
     "infv2_pipeline_destroy", "infv2_sparse_attn_rows", "infv2_decode_attn",
     "infv2_selftest_exp2", "infv2_varlen_kernel_offsets", "infv2_compress_k_varlen",
     "infv2_block_scores_varlen", "infv2_select_topk_varlen", "infv2_sparse_attn_varlen",
-    "infv2_dense_attn_varlen",
+    "infv2_dense_attn_varlen", "infv2_get_device_status",
 ]
 
 
@@ -70,6 +70,7 @@ def lib():
         L.infv2_status_string.restype = ctypes.c_char_p
         L.infv2_num_kernels.argtypes = [P, i]
         L.infv2_device_status.argtypes = [vp]
+        L.infv2_get_device_status.argtypes = [vp]
         L.infv2_compress_k.argtypes = [P, vp, i, vp, vp]
         L.infv2_block_scores.argtypes = [P, vp, vp, i, i, i, vp, i, vp, vp]
         L.infv2_select_topk.argtypes = [P, vp, i, i, i, i, vp, vp]
@@ -167,6 +168,11 @@ def infv2_check_params(p: Params) -> int:
 
 def infv2_device_status(stream=None) -> int:
     return lib().infv2_device_status(_stream(stream))
+
+
+def infv2_get_device_status(stream=None) -> int:
+    """infv2_device_status under its second name."""
+    return lib().infv2_get_device_status(_stream(stream))
 
 
 def infv2_compress_k(p: Params, k: torch.Tensor, kc1: torch.Tensor | None = None, stream=None):
